@@ -1,0 +1,170 @@
+"""Plain fp64 CPU oracle for the gated delta rule -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline / reference
+arm of ``bench.py`` may import this package.  The product library
+(``gated_deltanet_chunk_b200``) never imports it, and this package never imports
+the product library: the two share no code.
+
+The arithmetic lives in ``gdn_oracle.c`` (built to ``liboracle.so`` with gcc,
+``-O2 -fopenmp``; no fast-math, so every operation is a plain IEEE fp64 op).
+This module only marshals arrays:
+
+* :func:`recurrent` -- the definition: the token-by-token gated delta rule of
+  the "手撕Qwen3-Next" walkthrough, section 5(2) (torch_recurrent_gated_delta_rule).
+* :func:`chunk_form` -- the same walkthrough's chunkwise algorithm, section
+  5(1) steps a-g, with a generic chunk size.  Used only to pin the two forms
+  against each other.
+* :func:`chunk_prepare` -- the intra-chunk quantities of one chunk (gate
+  cumsum, decay mask, A, T = (I - A)^-1, U, W), for the inverse and similarity
+  pins.
+
+Inputs may be numpy arrays or CPU torch tensors of any float dtype (bf16
+included); they are upcast exactly to fp64.  Outputs are fp64 numpy arrays.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gdn_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+# tests/test_oracle_mutants.py points this at deliberately broken builds
+_LIB_OVERRIDE = os.environ.get("GDN_ORACLE_LIB_OVERRIDE")
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``gdn_oracle.c`` into ``liboracle.so`` (gcc, fp64, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp%d" % os.getpid()
+        subprocess.check_call(
+            ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-Wall",
+             "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        if _LIB_OVERRIDE:
+            lib = ctypes.CDLL(_LIB_OVERRIDE)
+        else:
+            build()
+            lib = ctypes.CDLL(_LIB)
+        dp = ctypes.POINTER(ctypes.c_double)
+        ip = ctypes.POINTER(ctypes.c_int32)
+        i = ctypes.c_int
+        lib.oracle_recurrent.argtypes = [i, ip, i, i, i, i, dp, dp, dp, dp, dp, dp, i,
+                                         ctypes.c_double, dp, dp]
+        lib.oracle_recurrent.restype = i
+        lib.oracle_chunk_form.argtypes = [i, ip, i, i, i, i, i, dp, dp, dp, dp, dp, dp, i,
+                                          ctypes.c_double, dp, dp]
+        lib.oracle_chunk_form.restype = i
+        lib.oracle_chunk_prepare.argtypes = [i, i, i, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp]
+        lib.oracle_chunk_prepare.restype = i
+        _lib = lib
+    return _lib
+
+
+def _f64(x):
+    if x is None:
+        return None
+    if hasattr(x, "detach"):  # torch tensor (CPU); bf16 -> fp32 -> fp64 is exact
+        import torch
+        x = x.detach().to("cpu")
+        if x.dtype in (torch.bfloat16, torch.float16):
+            x = x.float()
+        x = x.double().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _i32(x):
+    if hasattr(x, "detach"):
+        x = x.detach().to("cpu").numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.int32))
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    if a.dtype == np.int32:
+        return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _shapes(q, v, cu):
+    T, nqk, dk = q.shape
+    nv, dv = v.shape[1], v.shape[2]
+    if cu is None:
+        cu = np.array([0, T], dtype=np.int32)
+    cu = _i32(cu)
+    return T, nqk, dk, nv, dv, cu
+
+
+def recurrent(q, k, v, g, beta, initial_state=None, cu_seqlens=None,
+              qk_l2norm=True, scale=0.0):
+    """Token-loop definition.  Returns ``(out [T,Nv,Dv], final_state [N,Nv,Dk,Dv])``."""
+    q, k, v, g, beta = (_f64(x) for x in (q, k, v, g, beta))
+    s0 = _f64(initial_state)
+    T, nqk, dk, nv, dv, cu = _shapes(q, v, cu_seqlens)
+    n = len(cu) - 1
+    out = np.zeros((T, nv, dv))
+    sf = np.zeros((n, nv, dk, dv))
+    rc = _load().oracle_recurrent(n, _ptr(cu), nqk, nv, dk, dv, _ptr(q), _ptr(k), _ptr(v),
+                                  _ptr(g), _ptr(beta), _ptr(s0), int(bool(qk_l2norm)),
+                                  float(scale), _ptr(out), _ptr(sf))
+    if rc:
+        raise ValueError("oracle_recurrent: bad arguments (code %d)" % rc)
+    return out, sf
+
+
+def chunk_form(q, k, v, g, beta, chunk_size, initial_state=None, cu_seqlens=None,
+               qk_l2norm=True, scale=0.0):
+    """Chunkwise algorithm with chunk size ``chunk_size``.  Same outputs as :func:`recurrent`."""
+    q, k, v, g, beta = (_f64(x) for x in (q, k, v, g, beta))
+    s0 = _f64(initial_state)
+    T, nqk, dk, nv, dv, cu = _shapes(q, v, cu_seqlens)
+    n = len(cu) - 1
+    out = np.zeros((T, nv, dv))
+    sf = np.zeros((n, nv, dk, dv))
+    rc = _load().oracle_chunk_form(n, _ptr(cu), nqk, nv, dk, dv, int(chunk_size), _ptr(q),
+                                   _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(s0),
+                                   int(bool(qk_l2norm)), float(scale), _ptr(out), _ptr(sf))
+    if rc:
+        raise ValueError("oracle_chunk_form: bad arguments (code %d)" % rc)
+    return out, sf
+
+
+def chunk_prepare(kh, v, g, beta):
+    """Intra-chunk quantities of one chunk of already-normalised keys ``kh [C,Dk]``.
+
+    Returns a dict with ``gcum [C]``, ``gamma [C,C]``, ``A [C,C]``, ``T [C,C]``,
+    ``U [C,Dv]`` and ``W [C,Dk]``.
+    """
+    kh, v, g, beta = (_f64(x) for x in (kh, v, g, beta))
+    C, dk = kh.shape
+    dv = v.shape[1]
+    res = {"gcum": np.zeros(C), "gamma": np.zeros((C, C)), "A": np.zeros((C, C)),
+           "T": np.zeros((C, C)), "U": np.zeros((C, dv)), "W": np.zeros((C, dk))}
+    rc = _load().oracle_chunk_prepare(C, dk, dv, _ptr(kh), _ptr(v), _ptr(g), _ptr(beta),
+                                      *(_ptr(res[x]) for x in ("gcum", "gamma", "A", "T", "U", "W")))
+    if rc:
+        raise ValueError("oracle_chunk_prepare: bad arguments (code %d)" % rc)
+    return res
+
+
+def num_threads() -> int:
+    """Threads the OpenMP oracle uses (OMP_NUM_THREADS, else the CPU affinity set)."""
+    env = os.environ.get("OMP_NUM_THREADS")
+    if env and env.isdigit():
+        return int(env)
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
