@@ -1,0 +1,374 @@
+"""Throughput of the chunked gated delta rule (prefill) and the decode step on B200.
+
+One bench step = one gdn_chunk_fwd over the long-context prefill workload
+(2 sequences x 32768 tokens, Nqk = 16, Nv = 32, Dk = Dv = 128, chunk 64,
+bf16 q/k/v/out, fp32 g/beta/state, zero initial state), inputs resident in HBM.
+The decode workload (256 sequences x 1024 steps, same heads, fp32 state
+[256, 32, 128, 128] carried in place) is timed in the same run and reported
+under "decode".
+
+Prints ONE JSON line on rank 0.  Multi-GPU runs are independent replicas (each
+rank owns its own sequences; no collective on the data path): weak scaling.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--no-decode] [--no-e2e] [--no-cpu-baseline]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GDN chunked-fwd tokens/s (Nv=32,D=128) & decode tok/s; % of B200 roofline"
+PREFILL = "long_bf16_nv32"
+DECODE = "decode_bf16_nv32"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# --------------------------------------------------------------------------- accounting
+def prefill_bytes(T, nqk, nv, dk, dv, n, esz, s0=False, sf=True):
+    """Algorithmic bytes of one gdn_chunk_fwd: inputs read once, outputs written once."""
+    b = T * nqk * dk * esz * 2 + T * nv * dv * esz * 2 + T * nv * 4 * 2 + (n + 1) * 4
+    b += (n * nv * dk * dv * 4) * (int(s0) + int(sf))
+    return b
+
+
+def prefill_flops(T_per_seq, n, nv, C, D):
+    """(dense, triangular) FLOPs: per chunk-head 10C^2D + 6CD^2 + C^3/3, and 5C^2D + 6CD^2 + C^3/3."""
+    chunks = n * nv * ((T_per_seq + C - 1) // C)
+    dense = 10 * C * C * D + 6 * C * D * D + C ** 3 / 3
+    tri = 5 * C * C * D + 6 * C * D * D + C ** 3 / 3
+    return chunks * dense, chunks * tri
+
+
+def decode_bytes(n, nqk, nv, dk, dv, esz):
+    return n * nv * dk * dv * 4 * 2 + n * (2 * nqk * dk + 2 * nv * dv) * esz + n * nv * 4 * 2
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running (read-only)."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, index, period=0.02):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period, self.index = period, index
+        self._stop = threading.Event()
+        self._thread = None
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        except Exception:
+            self._nv = None
+        return self
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                mask = self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def summary(self):
+        return {"sm_mhz": (statistics.median(self.samples) if self.samples else None),
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------- distributed
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return world, rank, local  # rank 0 alone runs the CPU oracle; no process group
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world, device=None):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], device=device or "cpu", dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------- CPU oracle timing
+def time_oracle(w, T_sample, heads=None):
+    """Wall time of the fp64 oracle over the first T_sample tokens of each sequence."""
+    import torch
+
+    import oracle
+    cu = w["cu_seqlens"].tolist()
+    idx = torch.cat([torch.arange(cu[n], min(cu[n] + T_sample, cu[n + 1])) for n in range(len(cu) - 1)])
+    lens = [min(T_sample, cu[n + 1] - cu[n]) for n in range(len(cu) - 1)]
+    sub = {k: w[k][idx] for k in ("q", "k", "v", "g", "beta")}
+    cus = torch.tensor([0] + list(torch.cumsum(torch.tensor(lens), 0).tolist()), dtype=torch.int32)
+    # conversion to fp64 arrays happens before the clock starts
+    q, k, v, g, beta = (oracle._f64(sub[x]) for x in ("q", "k", "v", "g", "beta"))
+    t0 = time.perf_counter()
+    oracle.recurrent(q, k, v, g, beta, None, cus)
+    dt = time.perf_counter() - t0
+    return sum(lens), dt
+
+
+# --------------------------------------------------------------------------- main
+def run_ours(args, world, rank, local):
+    import torch
+
+    import gated_deltanet_chunk_b200 as gdn
+    import workloads as W
+
+    dev = torch.device("cuda", local)
+    peaks, peak_src = load_peaks()
+    wl = W.WORKLOADS[PREFILL]
+    host = W.make_workload(PREFILL, seed=2 + rank)          # each rank: its own sequences
+    n, T, nqk, nv, D, C = wl.num_seqs, host["T"], wl.nqk, wl.nv, wl.d, wl.chunk
+    d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in host.items()}
+    out = torch.empty(T, nv, D, dtype=torch.bfloat16, device=dev)
+    sf = torch.empty(n, nv, D, D, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        gdn.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], None, None, chunk_size=C,
+                      out=out, final_state=sf, num_seqs=n)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for i in range(args.steps):
+            evs[i][0].record(stream)
+            step()
+            evs[i][1].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end), world, dev)
+    per_launch_ms = [a.elapsed_time(b) for a, b in evs]
+    kern_ms = statistics.mean(per_launch_ms)
+    ms_per_step = total_ms / args.steps
+    tokens_all = T * world * args.steps
+    value = tokens_all / (total_ms / 1e3)
+
+    bytes_alg = prefill_bytes(T, nqk, nv, D, D, n, 2, s0=False, sf=True)
+    fl_dense, fl_tri = prefill_flops(T // n, n, nv, C, D)
+    achieved_gbs = bytes_alg / (kern_ms / 1e3) / 1e9
+    peak_key = "hbm_gbs"
+    res = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic (seeded; workloads/)",
+        "config": {"workload": PREFILL, "num_seqs": n, "seq_len": T // n, "nqk": nqk, "nv": nv,
+                   "dk": D, "dv": D, "chunk": C, "io": "bf16", "state": "fp32",
+                   "initial_state": "zeros", "l2": "inputs 1.63 GB > 126 MB L2; no flush",
+                   "parallelism": "replicas x%d" % world},
+        "gpu_launches": args.steps,
+        "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks[peak_key],
+                     "unit": "GB/s", "frac": achieved_gbs / peaks[peak_key], "traffic": None,
+                     "peak_source": peak_src, "alg_bytes_per_launch": bytes_alg,
+                     "kernel_ms": kern_ms,
+                     "tensor_tflops_tri": fl_tri / (kern_ms / 1e3) / 1e12,
+                     "tensor_frac_tri": fl_tri / (kern_ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+                     "flops_tri_per_launch": fl_tri, "flops_dense_per_launch": fl_dense,
+                     "roofline_time_ms": max(bytes_alg / (peaks["hbm_gbs"] * 1e9),
+                                             fl_tri / (peaks["bf16_tflops"] * 1e12)) * 1e3},
+        "clocks": clk.summary(),
+    }
+    # e2e: same call with host buffers (pinned), copies inside the timed region
+    if not args.no_e2e:
+        hp = {k: host[k].pin_memory() for k in ("q", "k", "v", "g", "beta")}
+        ho = torch.empty(T, nv, D, dtype=torch.bfloat16).pin_memory()
+        hs = torch.empty(n, nv, D, D, dtype=torch.float32).pin_memory()
+        bi = sum(t.numel() * t.element_size() for t in hp.values())
+        bo = ho.numel() * 2 + hs.numel() * 4
+
+        def e2e_step():
+            for k_ in hp:
+                d[k_].copy_(hp[k_], non_blocking=True)
+            step()
+            ho.copy_(out, non_blocking=True)
+            hs.copy_(sf, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        e_steps = max(3, min(args.steps, 10))
+        barrier(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        e_ms = max_over_ranks(a.elapsed_time(b), world, dev)
+        res["e2e"] = {"value": T * world * e_steps / (e_ms / 1e3), "unit": "tokens/s",
+                      "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "steps": e_steps}
+    del d
+    torch.cuda.empty_cache()
+    if not args.no_decode:
+        res["decode"] = run_decode(args, world, rank, dev, stream, peaks, peak_src)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        tok, dt = time_oracle(host, args.cpu_sample_tokens)
+        res["cpu_baseline"] = {"value": tok / dt, "unit": "tokens/s", "cores": oracle.num_threads(),
+                               "kind": "oracle",
+                               "sample": "fp64 token loop over the first %d tokens of each of the %d "
+                                         "sequences, all %d v-heads (%.1f s wall)"
+                                         % (args.cpu_sample_tokens, n, nv, dt)}
+    return res
+
+
+def run_decode(args, world, rank, dev, stream, peaks, peak_src):
+    import torch
+
+    import gated_deltanet_chunk_b200 as gdn
+    import workloads as W
+    wl = W.WORKLOADS[DECODE]
+    steps = wl.steps
+    d = W.make_decode(num_seqs=wl.num_seqs, steps=steps, nqk=wl.nqk, nv=wl.nv, d=wl.d, io=wl.io,
+                      seed=4 + rank, device=str(dev))
+    state = d["initial_state"]
+    out = torch.empty(wl.num_seqs, wl.nv, wl.d, dtype=torch.bfloat16, device=dev)
+
+    def run(n_steps):
+        for t in range(n_steps):
+            gdn.recurrent_step(d["q"][t], d["k"][t], d["v"][t], d["g"][t], d["beta"][t], state, out=out)
+
+    run(min(steps, 32))
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    run(steps)
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    ms = max_over_ranks(a.elapsed_time(b), world, dev)
+    per_step_ms = ms / steps
+    byts = decode_bytes(wl.num_seqs, wl.nqk, wl.nv, wl.d, wl.d, 2)
+    gbs = byts / (per_step_ms / 1e3) / 1e9
+    return {"value": wl.num_seqs * steps * world / (ms / 1e3), "unit": "tokens/s",
+            "workload": DECODE, "steps": steps, "ms_per_step": per_step_ms, "gpu_launches": steps,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "traffic": None, "peak_source": peak_src,
+                         "alg_bytes_per_launch": byts}}
+
+
+def run_reference(args, world, rank):
+    """The fp64 CPU oracle as the reference arm, on a bounded sample of the same workload."""
+    import oracle
+    import workloads as W
+    if rank != 0:
+        return None
+    wl = W.WORKLOADS[PREFILL]
+    host = W.make_workload(PREFILL, seed=2)
+    for _ in range(args.warmup):
+        time_oracle(host, args.ref_sample_tokens)
+    tot_tok, tot_s = 0, 0.0
+    for _ in range(args.steps):
+        tok, dt = time_oracle(host, args.ref_sample_tokens)
+        tot_tok += tok
+        tot_s += dt
+    value = tot_tok / tot_s
+    sample = ("fp64 token loop over the first %d tokens of each of the %d sequences, all %d v-heads, "
+              "per step" % (args.ref_sample_tokens, wl.num_seqs, wl.nv))
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_s / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded; workloads/)",
+            "config": {"workload": PREFILL, "num_seqs": wl.num_seqs, "seq_len": wl.seq_len,
+                       "nqk": wl.nqk, "nv": wl.nv, "dk": wl.d, "dv": wl.d, "chunk": wl.chunk,
+                       "io": "bf16", "parallelism": "host cores"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-tokens", type=int, default=4096)
+    ap.add_argument("--ref-sample-tokens", type=int, default=512)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        res = run_reference(args, world, rank)
+    else:
+        res = run_ours(args, world, rank, local)
+    if rank == 0 and res is not None:
+        print(json.dumps(res), flush=True)
+    if world > 1 and args.impl == "ours":
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

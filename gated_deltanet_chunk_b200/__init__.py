@@ -1,0 +1,136 @@
+"""Gated delta rule (Gated DeltaNet core) on B200: thin Python binding of libgdn.so.
+
+Every step of the computation runs in the CUDA kernels of ``libgdn.so``; this
+module only marshals torch CUDA tensors into the C ABI of ``include/gdn.h``
+(pointers, sizes, the current stream) and allocates outputs when the caller
+does not pass them.  There is no CPU or PyTorch fallback: if the library is
+missing the import fails, and if a call is rejected it raises ``GdnError``.
+
+Functions
+---------
+chunk_fwd(q, k, v, g, beta, ...)       -> (out, final_state)   prefill, gdn_chunk_fwd
+recurrent_step(q, k, v, g, beta, state, ...) -> out            decode, gdn_recurrent_step
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgdn.so")
+
+GDN_OK = 0
+STATUS_NAMES = {0: "GDN_OK", -1: "GDN_ERR_NULL", -2: "GDN_ERR_SHAPE", -3: "GDN_ERR_ALIGN",
+                -4: "GDN_ERR_ALIAS", -5: "GDN_ERR_CUDA", -6: "GDN_ERR_DEVICE",
+                -7: "GDN_ERR_DEVICE_TIMEOUT"}
+KERNELS = {"auto": 0, "simt": 1, "tc": 2}
+DTYPE_F32, DTYPE_BF16 = 0, 1
+
+
+class GdnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__("%s failed: %s" % (what, lib().gdn_status_string(status).decode()))
+
+
+class GdnParams(ctypes.Structure):
+    _fields_ = [("num_qk_heads", ctypes.c_int32), ("num_v_heads", ctypes.c_int32),
+                ("head_k_dim", ctypes.c_int32), ("head_v_dim", ctypes.c_int32),
+                ("io_dtype", ctypes.c_int32), ("qk_l2norm", ctypes.c_int32),
+                ("scale", ctypes.c_float), ("kernel", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libgdn.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                "libgdn.so is not built (expected at %s); run "
+                "`python -m gated_deltanet_chunk_b200.build`" % LIB_PATH)
+        L = ctypes.CDLL(LIB_PATH)
+        vp, fp, ip = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p
+        L.gdn_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, fp, ip, ctypes.c_int32, ctypes.c_int64,
+                                    ctypes.c_int32, vp, fp, ctypes.POINTER(GdnParams), vp]
+        L.gdn_chunk_fwd.restype = ctypes.c_int
+        L.gdn_recurrent_step.argtypes = [vp, vp, vp, fp, fp, fp, vp, ctypes.c_int32,
+                                         ctypes.POINTER(GdnParams), vp]
+        L.gdn_recurrent_step.restype = ctypes.c_int
+        L.gdn_device_status.argtypes = [vp]
+        L.gdn_device_status.restype = ctypes.c_int
+        L.gdn_status_string.argtypes = [ctypes.c_int]
+        L.gdn_status_string.restype = ctypes.c_char_p
+        L.gdn_version.argtypes = []
+        L.gdn_version.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def make_params(nqk, nv, dk, dv, io_bf16, qk_l2norm=True, scale=0.0, kernel="auto") -> GdnParams:
+    return GdnParams(int(nqk), int(nv), int(dk), int(dv), DTYPE_BF16 if io_bf16 else DTYPE_F32,
+                     1 if qk_l2norm else 0, float(scale), KERNELS[kernel])
+
+
+def chunk_fwd(q, k, v, g, beta, initial_state=None, cu_seqlens=None, chunk_size=64,
+              out=None, final_state=None, output_final_state=True, num_seqs=None,
+              qk_l2norm=True, scale=0.0, kernel="auto", stream=None, check=True):
+    """Chunked gated delta rule over a packed batch (``gdn_chunk_fwd``).
+
+    q, k [T, Nqk, Dk] and v [T, Nv, Dv] (bf16 or fp32, CUDA, contiguous);
+    g, beta [T, Nv] fp32; initial_state [N, Nv, Dk, Dv] fp32 or None;
+    cu_seqlens [N+1] int32 or None (then ``num_seqs`` equal sequences, default 1).
+    Returns ``(out, final_state)``; final_state is None when not requested.
+    """
+    import torch
+    T, nqk, dk = q.shape
+    nv, dv = v.shape[1], v.shape[2]
+    n = (cu_seqlens.numel() - 1) if cu_seqlens is not None else (num_seqs or 1)
+    if out is None:
+        out = torch.empty((T, nv, dv), dtype=v.dtype, device=v.device)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((n, nv, dk, dv), dtype=torch.float32, device=v.device)
+    p = make_params(nqk, nv, dk, dv, q.dtype == torch.bfloat16, qk_l2norm, scale, kernel)
+    rc = lib().gdn_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state),
+                             _ptr(cu_seqlens), int(n), int(T), int(chunk_size), _ptr(out),
+                             _ptr(final_state), ctypes.byref(p), _stream(stream))
+    if check and rc != GDN_OK:
+        raise GdnError(rc, "gdn_chunk_fwd")
+    return out, final_state
+
+
+def recurrent_step(q, k, v, g, beta, state, out=None, qk_l2norm=True, scale=0.0, stream=None,
+                   check=True):
+    """One decode token per sequence (``gdn_recurrent_step``); ``state`` is updated in place.
+
+    q, k [N, Nqk, Dk], v [N, Nv, Dv], g, beta [N, Nv], state [N, Nv, Dk, Dv] fp32.
+    Returns out [N, Nv, Dv].
+    """
+    import torch
+    N, nqk, dk = q.shape
+    nv, dv = v.shape[1], v.shape[2]
+    if out is None:
+        out = torch.empty((N, nv, dv), dtype=v.dtype, device=v.device)
+    p = make_params(nqk, nv, dk, dv, q.dtype == torch.bfloat16, qk_l2norm, scale)
+    rc = lib().gdn_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state),
+                                  _ptr(out), int(N), ctypes.byref(p), _stream(stream))
+    if check and rc != GDN_OK:
+        raise GdnError(rc, "gdn_recurrent_step")
+    return out
+
+
+def device_status(stream=None) -> int:
+    """Synchronise the stream and return the library's device status (``gdn_device_status``)."""
+    return lib().gdn_device_status(_stream(stream))

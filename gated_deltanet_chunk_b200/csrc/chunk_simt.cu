@@ -1,0 +1,387 @@
+// chunk_simt.cu -- chunked gated-delta-rule forward with fp32 CUDA-core arithmetic.
+//
+// This is the kernel for the fp32 io path (and any shape the tensor-core kernel
+// does not take).  It follows the chunkwise algorithm of the "手撕Qwen3-Next"
+// walkthrough, section 一(一)5(1) (torch_chunk_gated_delta_rule), with two
+// re-associations that avoid materialising W and the output attention's
+// separate U term:
+//
+//   V' = U - W S = T diag(beta) (V - diag(exp(gcum)) K S)          (step e/f)
+//   o  = diag(exp(gcum)) Q S + P V',  P = (Q K^T * Gamma), lower incl. diagonal
+//   S <- exp(g_last) S + (K * exp(g_last - gcum))^T V'
+//
+// where T = (I - A)^-1 is obtained by the walkthrough's row recursion (step d),
+// A = -strictLower(diag(beta) (K K^T * Gamma)), Gamma = exp(gcum_r - gcum_i)
+// for i <= r (mask before exp), gcum = in-chunk inclusive cumsum of g (step c).
+//
+// One CTA owns one (sequence, v-head, 32-column slice of Dv): the state
+// recurrence is separable in the Dv columns, so slices are independent.  The
+// CTA walks its sequence's chunks in order, keeping the fp32 state slice
+// [Dk x 32] in shared memory.  Rows past the sequence end behave as
+// q = k = v = g = beta = 0 (the walkthrough's zero padding), which leaves the
+// state unchanged.
+#include "gdn_common.cuh"
+#include "gdn_launch.h"
+
+namespace gdn {
+namespace simt {
+
+constexpr int kThreads = 256;
+constexpr int kDVS = 32;  // Dv columns per CTA
+
+template <int C, int DK>
+struct Smem {
+  static constexpr int AP = C + 1;                // padded pitch of A / T / P rows
+  static constexpr int kKhT = 0;                  // [DK][C] keys, transposed, swizzled
+  static constexpr int kQhT = kKhT + DK * C;      // [DK][C] queries, transposed, swizzled
+  static constexpr int kA = kQhT + DK * C;        // [C][AP] A, then T - I, then P
+  static constexpr int kS = kA + C * AP;          // [DK][kDVS] state slice
+  static constexpr int kV = kS + DK * kDVS;       // [C][kDVS] X, then V'
+  static constexpr int kGc = kV + C * kDVS;       // [C] gcum
+  static constexpr int kBeta = kGc + C;           // [C] beta
+  static constexpr int kEg = kBeta + C;           // [C] exp(gcum)
+  static constexpr int kEkl = kEg + C;            // [C] exp(g_last - gcum)
+  static constexpr int kTotal = kEkl + C;
+  static constexpr size_t kBytes = size_t(kTotal) * sizeof(float);
+  static_assert(kS % 4 == 0 && kV % 4 == 0, "float4 alignment");
+  static_assert(kBytes <= 232448, "shared memory budget");
+};
+
+// Transposed [D][C] tile with a 16-byte XOR swizzle: element (d, r).
+template <int C>
+__device__ __forceinline__ int swz(int d, int r) {
+  return d * C + ((((r >> 2) ^ (d & 7))) << 2) + (r & 3);
+}
+
+template <int C>
+__device__ __forceinline__ float4 ld4_t(const float* base, int d, int r0) {
+  return *reinterpret_cast<const float4*>(base + swz<C>(d, r0));
+}
+
+// A (IS_P = false):  A[r][i] = -beta_r (k_r . k_i) Gamma[r][i] for i < r, else 0.
+// P (IS_P = true):   P[r][i] = (q_r . k_i) Gamma[r][i] for i <= r, else 0.
+template <int C, int DK, bool IS_P>
+__device__ __forceinline__ void pair_matrix(float* sm, int tid) {
+  using L = Smem<C, DK>;
+  const float* X = sm + (IS_P ? L::kQhT : L::kKhT);
+  const float* Kt = sm + L::kKhT;
+  const float* gc = sm + L::kGc;
+  const float* bt = sm + L::kBeta;
+  float* A = sm + L::kA;
+  constexpr int NTC = C / 4;
+  for (int tile = tid; tile < NTC * NTC; tile += kThreads) {
+    const int r0 = (tile / NTC) * 4, i0 = (tile % NTC) * 4;
+    float acc[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+    if (i0 <= r0 + 3) {
+#pragma unroll 4
+      for (int d = 0; d < DK; ++d) {
+        const float4 x = ld4_t<C>(X, d, r0);
+        const float4 y = ld4_t<C>(Kt, d, i0);
+        const float xs[4] = {x.x, x.y, x.z, x.w};
+        const float ys[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+          for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(xs[a], ys[b], acc[a][b]);
+      }
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int r = r0 + a, i = i0 + b;
+        float val = 0.f;
+        if (IS_P ? (i <= r) : (i < r)) {
+          val = acc[a][b] * expf(gc[r] - gc[i]);  // masked before exp: gc[r] - gc[i] <= 0
+          if (!IS_P) val = -bt[r] * val;
+        }
+        A[r * L::AP + i] = val;
+      }
+  }
+}
+
+template <int C, int DK, typename IO>
+__global__ void __launch_bounds__(kThreads, 1) chunk_fwd_simt_kernel(ChunkArgs a) {
+  using L = Smem<C, DK>;
+  extern __shared__ __align__(16) float sm[];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int cslice = blockIdx.x * kDVS;  // first Dv column of this CTA
+  const int h = blockIdx.y;              // v-head
+  const int n = blockIdx.z;              // sequence
+  const int j = h / (a.nv / a.nqk);      // qk-head
+  const IO* q = static_cast<const IO*>(a.q);
+  const IO* k = static_cast<const IO*>(a.k);
+  const IO* v = static_cast<const IO*>(a.v);
+  IO* out = static_cast<IO*>(a.out);
+  const int dv = a.dv;
+  const int nv = a.nv, nqk = a.nqk;
+
+  int64_t seq_start, seq_end;
+  seq_bounds(a.cu, a.uniform_len, n, seq_start, seq_end);
+
+  float* S = sm + L::kS;
+  float* KhT = sm + L::kKhT;
+  float* QhT = sm + L::kQhT;
+  float* A = sm + L::kA;
+  float* V = sm + L::kV;
+  float* gc = sm + L::kGc;
+  float* bt = sm + L::kBeta;
+  float* eg = sm + L::kEg;
+  float* ekl = sm + L::kEkl;
+
+  const size_t state_off = ((size_t)n * nv + h) * (size_t)DK * dv;
+  for (int e = tid; e < DK * kDVS; e += kThreads) {
+    const int d = e / kDVS, c = e % kDVS;
+    S[e] = a.s0 ? a.s0[state_off + (size_t)d * dv + cslice + c] : 0.f;
+  }
+
+  for (int64_t c0 = seq_start; c0 < seq_end; c0 += C) {
+    __syncthreads();  // previous chunk fully consumed
+    // ---- load q, k rows; L2 norm (eps inside the root) and query scale ----
+    constexpr int PER = DK / 32;
+    for (int r = warp; r < C; r += kThreads / 32) {
+      const int64_t t = c0 + r;
+      const bool valid = t < seq_end;
+      float qv[PER], kv[PER];
+      float sq = 0.f, sk = 0.f;
+#pragma unroll
+      for (int e = 0; e < PER; ++e) {
+        const size_t off = ((size_t)t * nqk + j) * DK + lane * PER + e;
+        qv[e] = valid ? to_f32(q[off]) : 0.f;
+        kv[e] = valid ? to_f32(k[off]) : 0.f;
+        sq += qv[e] * qv[e];
+        sk += kv[e] * kv[e];
+      }
+      sq = warp_sum(sq);
+      sk = warp_sum(sk);
+      const float fq = (a.qk_l2norm ? 1.f / sqrtf(sq + kNormEps) : 1.f) * a.scale;
+      const float fk = a.qk_l2norm ? 1.f / sqrtf(sk + kNormEps) : 1.f;
+#pragma unroll
+      for (int e = 0; e < PER; ++e) {
+        const int d = lane * PER + e;
+        QhT[swz<C>(d, r)] = qv[e] * fq;
+        KhT[swz<C>(d, r)] = kv[e] * fk;
+      }
+    }
+    if (tid < C) {
+      const int64_t t = c0 + tid;
+      const bool valid = t < seq_end;
+      gc[tid] = valid ? a.g[(size_t)t * nv + h] : 0.f;
+      bt[tid] = valid ? a.beta[(size_t)t * nv + h] : 0.f;
+    }
+    __syncthreads();
+    // ---- in-chunk inclusive cumsum of g (one warp) ----
+    if (warp == 0) {
+      constexpr int PG = C / 32;
+      float loc[PG];
+      float run = 0.f;
+#pragma unroll
+      for (int e = 0; e < PG; ++e) {
+        run += gc[lane * PG + e];
+        loc[e] = run;
+      }
+      float incl = run;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      float excl = __shfl_up_sync(0xffffffffu, incl, 1);
+      if (lane == 0) excl = 0.f;
+#pragma unroll
+      for (int e = 0; e < PG; ++e) gc[lane * PG + e] = loc[e] + excl;
+    }
+    __syncthreads();
+    if (tid < C) {
+      const float glast = gc[C - 1];
+      eg[tid] = expf(gc[tid]);
+      ekl[tid] = expf(glast - gc[tid]);
+    }
+    // ---- A = -strictLower(diag(beta) (K K^T * Gamma)) ----
+    pair_matrix<C, DK, false>(sm, tid);
+    __syncthreads();
+    // ---- T - I by the row recursion  Tt_i = A_i + A_i Tt_{<i} ----
+    {
+      constexpr int TPJ = kThreads / C;  // threads per column
+      const int jc = tid / TPJ, part = tid % TPJ;
+      for (int i = 1; i < C; ++i) {
+        float val = 0.f;
+        if (jc < i)
+          for (int m = jc + 1 + part; m < i; m += TPJ) val = fmaf(A[i * L::AP + m], A[m * L::AP + jc], val);
+#pragma unroll
+        for (int o = 1; o < TPJ; o <<= 1) val += __shfl_xor_sync(0xffffffffu, val, o);
+        __syncthreads();
+        if (jc < i && part == 0) A[i * L::AP + jc] += val;
+        __syncthreads();
+      }
+    }
+    // ---- X = diag(beta) (V - diag(exp(gcum)) K S) ----
+    constexpr int NTV = (C / 4) * (kDVS / 4);
+    for (int tile = tid; tile < NTV; tile += kThreads) {
+      const int r0 = (tile / (kDVS / 4)) * 4, cc0 = (tile % (kDVS / 4)) * 4;
+      float acc[4][4] = {};
+#pragma unroll 4
+      for (int d = 0; d < DK; ++d) {
+        const float4 x = ld4_t<C>(KhT, d, r0);
+        const float4 y = *reinterpret_cast<const float4*>(S + d * kDVS + cc0);
+        const float xs[4] = {x.x, x.y, x.z, x.w};
+        const float ys[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+        for (int aa = 0; aa < 4; ++aa)
+#pragma unroll
+          for (int b = 0; b < 4; ++b) acc[aa][b] = fmaf(xs[aa], ys[b], acc[aa][b]);
+      }
+#pragma unroll
+      for (int aa = 0; aa < 4; ++aa) {
+        const int r = r0 + aa;
+        const int64_t t = c0 + r;
+        const bool valid = t < seq_end;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const float vv = valid ? to_f32(v[((size_t)t * nv + h) * dv + cslice + cc0 + b]) : 0.f;
+          V[r * kDVS + cc0 + b] = bt[r] * (vv - eg[r] * acc[aa][b]);
+        }
+      }
+    }
+    __syncthreads();
+    // ---- V' = T X = X + (T - I) X  (one 4x4 tile per thread: NTV <= kThreads) ----
+    {
+      static_assert(NTV <= kThreads, "one V' tile per thread");
+      float acc[4][4];
+      const int r0 = (tid / (kDVS / 4)) * 4, cc0 = (tid % (kDVS / 4)) * 4;
+      if (tid < NTV) {
+#pragma unroll
+        for (int aa = 0; aa < 4; ++aa) {
+          const float4 x = *reinterpret_cast<const float4*>(V + (r0 + aa) * kDVS + cc0);
+          acc[aa][0] = x.x; acc[aa][1] = x.y; acc[aa][2] = x.z; acc[aa][3] = x.w;
+        }
+        for (int i = 0; i < r0 + 3; ++i) {
+          const float4 y = *reinterpret_cast<const float4*>(V + i * kDVS + cc0);
+          const float ys[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+          for (int aa = 0; aa < 4; ++aa) {
+            const float t_ri = A[(r0 + aa) * L::AP + i];  // zero for i >= r
+#pragma unroll
+            for (int b = 0; b < 4; ++b) acc[aa][b] = fmaf(t_ri, ys[b], acc[aa][b]);
+          }
+        }
+      }
+      __syncthreads();
+      if (tid < NTV) {
+#pragma unroll
+        for (int aa = 0; aa < 4; ++aa)
+          *reinterpret_cast<float4*>(V + (r0 + aa) * kDVS + cc0) =
+              make_float4(acc[aa][0], acc[aa][1], acc[aa][2], acc[aa][3]);
+      }
+    }
+    __syncthreads();
+    // ---- P = (Q K^T * Gamma), lower including the diagonal ----
+    pair_matrix<C, DK, true>(sm, tid);
+    __syncthreads();
+    // ---- o = diag(exp(gcum)) Q S + P V' ----
+    for (int tile = tid; tile < NTV; tile += kThreads) {
+      const int r0 = (tile / (kDVS / 4)) * 4, cc0 = (tile % (kDVS / 4)) * 4;
+      float acc[4][4] = {};
+#pragma unroll 4
+      for (int d = 0; d < DK; ++d) {
+        const float4 x = ld4_t<C>(QhT, d, r0);
+        const float4 y = *reinterpret_cast<const float4*>(S + d * kDVS + cc0);
+        const float xs[4] = {x.x, x.y, x.z, x.w};
+        const float ys[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+        for (int aa = 0; aa < 4; ++aa)
+#pragma unroll
+          for (int b = 0; b < 4; ++b) acc[aa][b] = fmaf(xs[aa], ys[b], acc[aa][b]);
+      }
+#pragma unroll
+      for (int aa = 0; aa < 4; ++aa)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[aa][b] *= eg[r0 + aa];
+      for (int i = 0; i <= r0 + 3 && i < C; ++i) {
+        const float4 y = *reinterpret_cast<const float4*>(V + i * kDVS + cc0);
+        const float ys[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+        for (int aa = 0; aa < 4; ++aa) {
+          const float p = A[(r0 + aa) * L::AP + i];  // zero for i > r
+#pragma unroll
+          for (int b = 0; b < 4; ++b) acc[aa][b] = fmaf(p, ys[b], acc[aa][b]);
+        }
+      }
+#pragma unroll
+      for (int aa = 0; aa < 4; ++aa) {
+        const int64_t t = c0 + r0 + aa;
+        if (t < seq_end) {
+          IO* orow = out + ((size_t)t * nv + h) * dv + cslice + cc0;
+#pragma unroll
+          for (int b = 0; b < 4; ++b) orow[b] = from_f32<IO>(acc[aa][b]);
+        }
+      }
+    }
+    __syncthreads();
+    // ---- S <- exp(g_last) S + (K * exp(g_last - gcum))^T V' ----
+    {
+      const float decay = expf(gc[C - 1]);
+      constexpr int NTS = (DK / 4) * (kDVS / 4);
+      for (int tile = tid; tile < NTS; tile += kThreads) {
+        const int d0 = (tile / (kDVS / 4)) * 4, cc0 = (tile % (kDVS / 4)) * 4;
+        float acc[4][4] = {};
+        for (int r = 0; r < C; ++r) {
+          const float w = ekl[r];
+          const float4 y = *reinterpret_cast<const float4*>(V + r * kDVS + cc0);
+          const float ys[4] = {y.x * w, y.y * w, y.z * w, y.w * w};
+#pragma unroll
+          for (int aa = 0; aa < 4; ++aa) {
+            const float kk = KhT[swz<C>(d0 + aa, r)];
+#pragma unroll
+            for (int b = 0; b < 4; ++b) acc[aa][b] = fmaf(kk, ys[b], acc[aa][b]);
+          }
+        }
+#pragma unroll
+        for (int aa = 0; aa < 4; ++aa) {
+          float4* sp = reinterpret_cast<float4*>(S + (d0 + aa) * kDVS + cc0);
+          float4 s = *sp;
+          s.x = fmaf(s.x, decay, acc[aa][0]);
+          s.y = fmaf(s.y, decay, acc[aa][1]);
+          s.z = fmaf(s.z, decay, acc[aa][2]);
+          s.w = fmaf(s.w, decay, acc[aa][3]);
+          *sp = s;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (a.s_final) {
+    for (int e = tid; e < DK * kDVS; e += kThreads) {
+      const int d = e / kDVS, c = e % kDVS;
+      a.s_final[state_off + (size_t)d * dv + cslice + c] = S[e];
+    }
+  }
+}
+
+template <int C, int DK, typename IO>
+static cudaError_t launch_one(const ChunkArgs& a, cudaStream_t stream) {
+  auto kern = chunk_fwd_simt_kernel<C, DK, IO>;
+  const size_t smem = Smem<C, DK>::kBytes;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.dv / kDVS, a.nv, a.num_seqs);
+  kern<<<grid, kThreads, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace simt
+
+cudaError_t launch_chunk_simt(const ChunkArgs& a, int dk, int chunk, int io_bf16, cudaStream_t s) {
+  using bf = __nv_bfloat16;
+  if (dk == 64 && chunk == 64) return io_bf16 ? simt::launch_one<64, 64, bf>(a, s) : simt::launch_one<64, 64, float>(a, s);
+  if (dk == 64 && chunk == 128) return io_bf16 ? simt::launch_one<128, 64, bf>(a, s) : simt::launch_one<128, 64, float>(a, s);
+  if (dk == 128 && chunk == 64) return io_bf16 ? simt::launch_one<64, 128, bf>(a, s) : simt::launch_one<64, 128, float>(a, s);
+  if (dk == 128 && chunk == 128) return io_bf16 ? simt::launch_one<128, 128, bf>(a, s) : simt::launch_one<128, 128, float>(a, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace gdn

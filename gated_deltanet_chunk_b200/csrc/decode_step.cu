@@ -1,0 +1,138 @@
+// decode_step.cu -- one-token gated delta rule step (decode), state updated in place.
+//
+// The token recurrence of the "手撕Qwen3-Next" walkthrough, section
+// 一(一)5(2) (torch_recurrent_gated_delta_rule), for one token per sequence:
+//
+//   S <- alpha S (alpha = exp(g));  kv = S^T k_hat;  delta = beta (v - kv)
+//   S <- S + k_hat delta^T;         o = S^T q_hat
+//
+// The state is read once and written once.  With the decayed old state
+// D = alpha S_old, both reductions come from one pass over D:
+//   kv_c = sum_r D[r,c] k_r,    o_c = sum_r D[r,c] q_r + delta_c (k_hat . q_hat)
+// (the second is q^T (D + k delta^T)).  The kernel is bound by HBM: per
+// (sequence, v-head) it streams Dk*Dv*4 bytes in and out.
+//
+// One CTA of 256 threads owns one (sequence, v-head).  Thread (rg, cg) holds
+// 4 consecutive columns (one 16-byte vector) of DK/RG rows in registers, so
+// every state byte is loaded with a 128-bit streaming load before any
+// arithmetic starts and written back with a 128-bit streaming store.
+#include "gdn_common.cuh"
+#include "gdn_launch.h"
+
+namespace gdn {
+namespace decode {
+
+constexpr int kThreads = 256;
+
+template <int DK, int DV, typename IO>
+__global__ void __launch_bounds__(kThreads, 2) recurrent_step_kernel(StepArgs a) {
+  constexpr int CG = DV / 4;         // column groups of 4 fp32
+  constexpr int RG = kThreads / CG;  // row groups
+  constexpr int RPT = DK / RG;       // rows per thread
+  static_assert(RPT >= 1 && DK % RG == 0, "shape");
+  __shared__ float qh[DK], kh[DK];
+  __shared__ float red_k[RG][DV], red_q[RG][DV];
+  __shared__ __align__(16) float delta[DV];
+  __shared__ float kq_s;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int h = blockIdx.x, n = blockIdx.y;
+  const int j = h / (a.nv / a.nqk);
+  const int cg = tid % CG, rg = tid / CG;
+
+  float4* st = reinterpret_cast<float4*>(a.state + ((size_t)n * a.nv + h) * (size_t)DK * DV);
+  float4 s[RPT];
+#pragma unroll
+  for (int i = 0; i < RPT; ++i) s[i] = __ldcs(st + (size_t)(i * RG + rg) * CG + cg);
+
+  const float alpha = expf(a.g[(size_t)n * a.nv + h]);
+  const float bta = a.beta[(size_t)n * a.nv + h];
+
+  // q_hat, k_hat (warp 0: q, warp 1: k)
+  if (warp < 2) {
+    const IO* src = static_cast<const IO*>(warp == 0 ? a.q : a.k) + ((size_t)n * a.nqk + j) * DK;
+    constexpr int PER = DK / 32;
+    float x[PER];
+    float ss = 0.f;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+      x[e] = to_f32(src[lane * PER + e]);
+      ss += x[e] * x[e];
+    }
+    ss = warp_sum(ss);
+    float f = a.qk_l2norm ? 1.f / sqrtf(ss + kNormEps) : 1.f;
+    if (warp == 0) f *= a.scale;
+    float* dst = warp == 0 ? qh : kh;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) dst[lane * PER + e] = x[e] * f;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    float p = 0.f;
+    for (int d = lane; d < DK; d += 32) p += qh[d] * kh[d];
+    p = warp_sum(p);
+    if (lane == 0) kq_s = p;
+  }
+
+  // partial reductions of the decayed state over this thread's rows
+  float pk[4] = {0.f, 0.f, 0.f, 0.f}, pq[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int i = 0; i < RPT; ++i) {
+    const int r = i * RG + rg;
+    s[i].x *= alpha; s[i].y *= alpha; s[i].z *= alpha; s[i].w *= alpha;
+    const float kr = kh[r], qr = qh[r];
+    pk[0] = fmaf(s[i].x, kr, pk[0]); pk[1] = fmaf(s[i].y, kr, pk[1]);
+    pk[2] = fmaf(s[i].z, kr, pk[2]); pk[3] = fmaf(s[i].w, kr, pk[3]);
+    pq[0] = fmaf(s[i].x, qr, pq[0]); pq[1] = fmaf(s[i].y, qr, pq[1]);
+    pq[2] = fmaf(s[i].z, qr, pq[2]); pq[3] = fmaf(s[i].w, qr, pq[3]);
+  }
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    red_k[rg][cg * 4 + c] = pk[c];
+    red_q[rg][cg * 4 + c] = pq[c];
+  }
+  __syncthreads();
+  if (tid < DV) {
+    const int c = tid;
+    float kv = 0.f, qs = 0.f;
+#pragma unroll
+    for (int r = 0; r < RG; ++r) {
+      kv += red_k[r][c];
+      qs += red_q[r][c];
+    }
+    const size_t vo = ((size_t)n * a.nv + h) * DV + c;
+    const float dl = bta * (to_f32(static_cast<const IO*>(a.v)[vo]) - kv);
+    delta[c] = dl;
+    static_cast<IO*>(a.out)[vo] = from_f32<IO>(fmaf(dl, kq_s, qs));
+  }
+  __syncthreads();
+  const float4 dl = *reinterpret_cast<const float4*>(delta + cg * 4);
+#pragma unroll
+  for (int i = 0; i < RPT; ++i) {
+    const float kr = kh[i * RG + rg];
+    float4 o;
+    o.x = fmaf(kr, dl.x, s[i].x); o.y = fmaf(kr, dl.y, s[i].y);
+    o.z = fmaf(kr, dl.z, s[i].z); o.w = fmaf(kr, dl.w, s[i].w);
+    __stcs(st + (size_t)(i * RG + rg) * CG + cg, o);
+  }
+}
+
+template <int DK, int DV, typename IO>
+static cudaError_t launch_one(const StepArgs& a, cudaStream_t stream) {
+  dim3 grid(a.nv, a.num_seqs);
+  recurrent_step_kernel<DK, DV, IO><<<grid, kThreads, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace decode
+
+cudaError_t launch_recurrent_step(const StepArgs& a, int dk, int dv, int io_bf16, cudaStream_t s) {
+  using bf = __nv_bfloat16;
+  if (dk == 64 && dv == 64) return io_bf16 ? decode::launch_one<64, 64, bf>(a, s) : decode::launch_one<64, 64, float>(a, s);
+  if (dk == 64 && dv == 128) return io_bf16 ? decode::launch_one<64, 128, bf>(a, s) : decode::launch_one<64, 128, float>(a, s);
+  if (dk == 128 && dv == 64) return io_bf16 ? decode::launch_one<128, 64, bf>(a, s) : decode::launch_one<128, 64, float>(a, s);
+  if (dk == 128 && dv == 128) return io_bf16 ? decode::launch_one<128, 128, bf>(a, s) : decode::launch_one<128, 128, float>(a, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace gdn

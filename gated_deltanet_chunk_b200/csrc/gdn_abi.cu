@@ -1,0 +1,181 @@
+// gdn_abi.cu -- the extern "C" boundary of libgdn.so: argument validation,
+// kernel choice and launch on the caller's stream.  See include/gdn.h.
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/gdn.h"
+#include "gdn_common.cuh"
+#include "gdn_launch.h"
+
+#define GDN_API extern "C" __attribute__((visibility("default")))
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Range {
+  uintptr_t lo, hi;  // [lo, hi)
+};
+
+Range range_of(const void* p, size_t bytes) {
+  const uintptr_t lo = reinterpret_cast<uintptr_t>(p);
+  return Range{lo, lo + bytes};
+}
+
+bool overlap(Range a, Range b) {
+  if (a.lo == a.hi || b.lo == b.hi) return false;
+  return a.lo < b.hi && b.lo < a.hi;
+}
+
+// The library ships sm_100a code only: require a compute capability 10.0 device.
+int check_device() {
+  static int ok[kMaxDevices] = {0};  // 0 unknown, 1 ok, -1 bad
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GDN_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return GDN_ERR_DEVICE;
+  if (ok[dev] == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return GDN_ERR_CUDA;
+    ok[dev] = (major == 10 && minor == 0) ? 1 : -1;
+  }
+  return ok[dev] == 1 ? GDN_OK : GDN_ERR_DEVICE;
+}
+
+int check_params(const gdn_params_t* p) {
+  if (!p) return GDN_ERR_NULL;
+  if (p->num_qk_heads < 1 || p->num_v_heads < 1 || p->num_v_heads > 65535 ||
+      p->num_v_heads % p->num_qk_heads != 0)
+    return GDN_ERR_SHAPE;
+  if ((p->head_k_dim != 64 && p->head_k_dim != 128) || (p->head_v_dim != 64 && p->head_v_dim != 128))
+    return GDN_ERR_SHAPE;
+  if (p->io_dtype != GDN_DTYPE_F32 && p->io_dtype != GDN_DTYPE_BF16) return GDN_ERR_SHAPE;
+  if (p->kernel < GDN_KERNEL_AUTO || p->kernel > GDN_KERNEL_TC) return GDN_ERR_SHAPE;
+  if (!std::isfinite(p->scale)) return GDN_ERR_SHAPE;
+  return GDN_OK;
+}
+
+float resolve_scale(const gdn_params_t* p) {
+  return p->scale > 0.f ? p->scale : 1.0f / std::sqrt((float)p->head_k_dim);
+}
+
+}  // namespace
+
+GDN_API int gdn_version(void) { return (1 << 16) | 0; }
+
+GDN_API const char* gdn_status_string(int status) {
+  switch (status) {
+    case GDN_OK: return "GDN_OK";
+    case GDN_ERR_NULL: return "GDN_ERR_NULL: a required pointer is NULL";
+    case GDN_ERR_SHAPE: return "GDN_ERR_SHAPE: unsupported head count, head dim, chunk size or length";
+    case GDN_ERR_ALIGN: return "GDN_ERR_ALIGN: a tensor pointer is not 16-byte aligned";
+    case GDN_ERR_ALIAS: return "GDN_ERR_ALIAS: an output overlaps an input";
+    case GDN_ERR_CUDA: return "GDN_ERR_CUDA: a CUDA call or kernel launch failed";
+    case GDN_ERR_DEVICE: return "GDN_ERR_DEVICE: the current device is not compute capability 10.0";
+    case GDN_ERR_DEVICE_TIMEOUT: return "GDN_ERR_DEVICE_TIMEOUT: a bounded in-kernel wait expired";
+    default: return "GDN: unknown status";
+  }
+}
+
+GDN_API int gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
+                          const float* beta, const float* initial_state,
+                          const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                          int32_t chunk_size, void* out, float* final_state,
+                          const gdn_params_t* p, void* cuda_stream) {
+  int rc = check_params(p);
+  if (rc) return rc;
+  if (!q || !k || !v || !g || !beta || !out) return GDN_ERR_NULL;
+  if (num_seqs < 1 || num_seqs > 65535) return GDN_ERR_SHAPE;
+  if (total_tokens < 0 || total_tokens >= (int64_t(1) << 31)) return GDN_ERR_SHAPE;
+  if (chunk_size != 64 && chunk_size != 128) return GDN_ERR_SHAPE;
+  if (!cu_seqlens && total_tokens % num_seqs != 0) return GDN_ERR_SHAPE;
+  const void* ptrs[] = {q, k, v, g, beta, initial_state, cu_seqlens, out, final_state};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return GDN_ERR_ALIGN;
+
+  const size_t T = (size_t)total_tokens, N = (size_t)num_seqs;
+  const size_t esz = p->io_dtype == GDN_DTYPE_BF16 ? 2 : 4;
+  const size_t dk = p->head_k_dim, dv = p->head_v_dim;
+  const size_t nqk = p->num_qk_heads, nv = p->num_v_heads;
+  const Range rq = range_of(q, T * nqk * dk * esz), rk = range_of(k, T * nqk * dk * esz);
+  const Range rv = range_of(v, T * nv * dv * esz);
+  const Range rg = range_of(g, T * nv * 4), rb = range_of(beta, T * nv * 4);
+  const Range rs0 = initial_state ? range_of(initial_state, N * nv * dk * dv * 4) : Range{0, 0};
+  const Range rcu = cu_seqlens ? range_of(cu_seqlens, (N + 1) * 4) : Range{0, 0};
+  const Range ro = range_of(out, T * nv * dv * esz);
+  const Range rsf = final_state ? range_of(final_state, N * nv * dk * dv * 4) : Range{0, 0};
+  for (Range r : {rq, rk, rv, rg, rb, rs0, rcu, rsf})
+    if (overlap(ro, r)) return GDN_ERR_ALIAS;
+  for (Range r : {rq, rk, rv, rg, rb, rcu})
+    if (overlap(rsf, r)) return GDN_ERR_ALIAS;
+  if (final_state && initial_state && (const void*)final_state != (const void*)initial_state &&
+      overlap(rsf, rs0))
+    return GDN_ERR_ALIAS;
+
+  rc = check_device();
+  if (rc) return rc;
+
+  gdn::ChunkArgs a;
+  a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta;
+  a.s0 = initial_state; a.cu = cu_seqlens; a.out = out; a.s_final = final_state;
+  a.uniform_len = cu_seqlens ? 0 : (int32_t)(total_tokens / num_seqs);
+  a.num_seqs = num_seqs;
+  a.nqk = p->num_qk_heads; a.nv = p->num_v_heads; a.dv = p->head_v_dim;
+  a.qk_l2norm = p->qk_l2norm ? 1 : 0;
+  a.scale = resolve_scale(p);
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+
+  if (p->kernel == GDN_KERNEL_TC) return GDN_ERR_SHAPE;  // tensor-core kernel: not available for these shapes
+  cudaError_t e = gdn::launch_chunk_simt(a, p->head_k_dim, chunk_size,
+                                         p->io_dtype == GDN_DTYPE_BF16, stream);
+  return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+GDN_API int gdn_recurrent_step(const void* q, const void* k, const void* v, const float* g,
+                               const float* beta, float* state, void* out, int32_t num_seqs,
+                               const gdn_params_t* p, void* cuda_stream) {
+  int rc = check_params(p);
+  if (rc) return rc;
+  if (!q || !k || !v || !g || !beta || !state || !out) return GDN_ERR_NULL;
+  if (num_seqs < 1 || num_seqs > 65535) return GDN_ERR_SHAPE;
+  const void* ptrs[] = {q, k, v, g, beta, state, out};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return GDN_ERR_ALIGN;
+  const size_t N = (size_t)num_seqs;
+  const size_t esz = p->io_dtype == GDN_DTYPE_BF16 ? 2 : 4;
+  const size_t dk = p->head_k_dim, dv = p->head_v_dim;
+  const size_t nqk = p->num_qk_heads, nv = p->num_v_heads;
+  const Range rq = range_of(q, N * nqk * dk * esz), rk = range_of(k, N * nqk * dk * esz);
+  const Range rv = range_of(v, N * nv * dv * esz);
+  const Range rg = range_of(g, N * nv * 4), rb = range_of(beta, N * nv * 4);
+  const Range rs = range_of(state, N * nv * dk * dv * 4);
+  const Range ro = range_of(out, N * nv * dv * esz);
+  for (Range r : {rq, rk, rv, rg, rb, rs})
+    if (overlap(ro, r)) return GDN_ERR_ALIAS;
+  for (Range r : {rq, rk, rv, rg, rb})
+    if (overlap(rs, r)) return GDN_ERR_ALIAS;
+
+  rc = check_device();
+  if (rc) return rc;
+
+  gdn::StepArgs a;
+  a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.state = state; a.out = out;
+  a.num_seqs = num_seqs;
+  a.nqk = p->num_qk_heads; a.nv = p->num_v_heads;
+  a.qk_l2norm = p->qk_l2norm ? 1 : 0;
+  a.scale = resolve_scale(p);
+  cudaError_t e = gdn::launch_recurrent_step(a, p->head_k_dim, p->head_v_dim,
+                                             p->io_dtype == GDN_DTYPE_BF16,
+                                             static_cast<cudaStream_t>(cuda_stream));
+  return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+GDN_API int gdn_device_status(void* cuda_stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(cuda_stream));
+  if (e != cudaSuccess) return GDN_ERR_CUDA;
+  return GDN_OK;
+}

@@ -1,0 +1,76 @@
+// gdn_common.cuh -- small device helpers and the argument blocks shared by the
+// gated-delta-rule kernels of libgdn.so (sm_100a only).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gdn {
+
+constexpr float kNormEps = 1e-6f;  // L2 norm eps, inside the square root
+
+// Arguments of the chunked forward (gdn_chunk_fwd); pointers are device memory.
+struct ChunkArgs {
+  const void* q;             // [T, Nqk, Dk]
+  const void* k;             // [T, Nqk, Dk]
+  const void* v;             // [T, Nv, Dv]
+  const float* g;            // [T, Nv]
+  const float* beta;         // [T, Nv]
+  const float* s0;           // [N, Nv, Dk, Dv] or nullptr
+  const int32_t* cu;         // [N + 1] or nullptr (equal lengths)
+  void* out;                 // [T, Nv, Dv]
+  float* s_final;            // [N, Nv, Dk, Dv] or nullptr
+  int32_t uniform_len;       // sequence length when cu == nullptr
+  int32_t num_seqs;
+  int32_t nqk, nv, dv;
+  int32_t qk_l2norm;
+  float scale;
+};
+
+// Arguments of the one-token decode step (gdn_recurrent_step).
+struct StepArgs {
+  const void* q;     // [N, Nqk, Dk]
+  const void* k;     // [N, Nqk, Dk]
+  const void* v;     // [N, Nv, Dv]
+  const float* g;    // [N, Nv]
+  const float* beta; // [N, Nv]
+  float* state;      // [N, Nv, Dk, Dv] in place
+  void* out;         // [N, Nv, Dv]
+  int32_t num_seqs;
+  int32_t nqk, nv;
+  int32_t qk_l2norm;
+  float scale;
+};
+
+template <typename T> __device__ __forceinline__ float to_f32(T x);
+template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
+  return __bfloat162float(x);
+}
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);  // round to nearest even
+}
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+// Sequence bounds [start, end) of sequence n.
+__device__ __forceinline__ void seq_bounds(const int32_t* cu, int32_t uniform_len, int n,
+                                           int64_t& start, int64_t& end) {
+  if (cu) {
+    start = cu[n];
+    end = cu[n + 1];
+  } else {
+    start = (int64_t)n * uniform_len;
+    end = start + uniform_len;
+  }
+}
+
+}  // namespace gdn

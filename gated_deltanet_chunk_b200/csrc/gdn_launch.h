@@ -1,0 +1,16 @@
+// gdn_launch.h -- launchers of the libgdn.so kernels (host side, internal).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "gdn_common.cuh"
+
+namespace gdn {
+
+// fp32 CUDA-core chunked forward; dk in {64,128}, chunk in {64,128}, dv % 32 == 0.
+cudaError_t launch_chunk_simt(const ChunkArgs& a, int dk, int chunk, int io_bf16, cudaStream_t s);
+
+// One-token decode step; dk, dv in {64,128}.
+cudaError_t launch_recurrent_step(const StepArgs& a, int dk, int dv, int io_bf16, cudaStream_t s);
+
+}  // namespace gdn

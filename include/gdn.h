@@ -1,0 +1,145 @@
+/*
+ * gdn.h -- C ABI of libgdn.so: the gated delta rule (Gated DeltaNet core) on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation is the gated delta rule as defined by the "手撕Qwen3-Next"
+ * walkthrough (wkq9411.github.io, Code-Qwen3-Next), section 一(一)5
+ * "应用 Gated Delta Rule": per v-head, with state S in R^{Dk x Dv},
+ *
+ *     q_hat = q / sqrt(sum q^2 + 1e-6) * scale,   k_hat = k / sqrt(sum k^2 + 1e-6)
+ *     S <- S * exp(g_t)
+ *     delta = beta_t (v_t - S^T k_hat)            (S^T k_hat: the value k_hat retrieves)
+ *     S <- S + k_hat delta^T
+ *     o_t = S^T q_hat                              (after token t's own write)
+ *
+ * gdn_chunk_fwd computes it for whole sequences with the chunkwise algorithm of
+ * section 5(1) (prefill); gdn_recurrent_step advances every sequence by one
+ * token (decode, section 5(2)).  The L2 norm with eps inside the root follows
+ * the PyPTO-Gym "Qwen3Next 样例" README (数学公式); the packed [T, N, D] layout
+ * with cumulative sequence lengths follows its 参数说明 (act_seq_len).
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE memory owned by the caller, contiguous,
+ *     row-major, 16-byte aligned.  The library never allocates or frees.
+ *   - Calls are asynchronous on `cuda_stream` (a cudaStream_t; NULL = legacy
+ *     default stream) of the CURRENT device.
+ *   - The return value is GDN_OK or a negative gdn_status_t.  Arguments are
+ *     validated on the host before anything is launched; a rejected call
+ *     launches nothing and writes nothing.
+ *   - Numbers: g, beta and the states are fp32; q, k, v and out have the
+ *     dtype `io_dtype`.  Every accumulation is fp32.
+ *   - GQA: v-head h reads qk-head h / (Nv / Nqk)  (repeat_interleave of the
+ *     walkthrough, section 4).
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_NULL = -1,           /* a required pointer is NULL */
+    GDN_ERR_SHAPE = -2,          /* unsupported head count, head dim, chunk size or length */
+    GDN_ERR_ALIGN = -3,          /* a tensor pointer is not 16-byte aligned */
+    GDN_ERR_ALIAS = -4,          /* `out` overlaps an input, or `state` overlaps q/k/v/out */
+    GDN_ERR_CUDA = -5,           /* a CUDA runtime call or kernel launch failed */
+    GDN_ERR_DEVICE = -6,         /* the current device is not a compute capability 10.0 GPU */
+    GDN_ERR_DEVICE_TIMEOUT = -7  /* a bounded in-kernel wait expired (see gdn_device_status) */
+} gdn_status_t;
+
+typedef enum { GDN_DTYPE_F32 = 0, GDN_DTYPE_BF16 = 1 } gdn_dtype_t;
+
+/* Kernel family for gdn_chunk_fwd.  AUTO picks the tensor-core kernel where it
+ * applies (bf16 io, Dk = Dv = 128) and the SIMT kernel otherwise. */
+typedef enum { GDN_KERNEL_AUTO = 0, GDN_KERNEL_SIMT = 1, GDN_KERNEL_TC = 2 } gdn_kernel_t;
+
+/* Shapes and options shared by both calls. */
+typedef struct {
+    int32_t num_qk_heads;  /* Nqk >= 1 */
+    int32_t num_v_heads;   /* Nv >= 1, Nv % Nqk == 0 */
+    int32_t head_k_dim;    /* Dk in {64, 128} */
+    int32_t head_v_dim;    /* Dv in {64, 128} */
+    int32_t io_dtype;      /* gdn_dtype_t of q, k, v, out */
+    int32_t qk_l2norm;     /* 1: L2-normalise q and k in-kernel (eps 1e-6); 0: use as given */
+    float scale;           /* query scale; <= 0 selects 1/sqrt(Dk) */
+    int32_t kernel;        /* gdn_kernel_t; 0 = automatic */
+} gdn_params_t;
+
+/*
+ * gdn_chunk_fwd -- chunked prefill over a packed batch of N sequences.
+ *
+ * Walkthrough section 5(1) steps a-g (torch_chunk_gated_delta_rule), per
+ * sequence; the PyPTO README's fused chunk_gated_delta_rule interface.
+ *
+ *   q, k           [T, Nqk, Dk]  io_dtype
+ *   v              [T, Nv, Dv]   io_dtype
+ *   g, beta        [T, Nv]       fp32   (g = log of the decay, beta = write strength)
+ *   initial_state  [N, Nv, Dk, Dv] fp32 (Dk rows, Dv contiguous) or NULL for zeros
+ *   cu_seqlens     [N + 1] int32 device array: cu[0] = 0, non-decreasing, cu[N] = T;
+ *                  sequence n owns tokens [cu[n], cu[n+1]) and starts from
+ *                  initial_state[n].  NULL means N equal sequences of T / N
+ *                  tokens (T % N must be 0).  Contents are not validated.
+ *   num_seqs       N >= 1 (N <= 65535)
+ *   total_tokens   T >= 0 (T < 2^31)
+ *   chunk_size     C in {64, 128}: the chunk length of the chunkwise algorithm.
+ *                  Every sequence has its own chunk grid starting at cu[n]; its
+ *                  tail chunk is processed as if zero padded.  The result does
+ *                  not depend on C beyond rounding.
+ *   out            [T, Nv, Dv] io_dtype; must not overlap any input
+ *   final_state    [N, Nv, Dk, Dv] fp32 or NULL; may be the same buffer as
+ *                  initial_state (updated in place); other overlaps are rejected
+ *   p              shapes and options (see gdn_params_t)
+ *
+ * Zero-length sequences are allowed: their final_state equals their initial state.
+ */
+int gdn_chunk_fwd(const void *q, const void *k, const void *v,
+                  const float *g, const float *beta,
+                  const float *initial_state,
+                  const int32_t *cu_seqlens,
+                  int32_t num_seqs, int64_t total_tokens, int32_t chunk_size,
+                  void *out, float *final_state,
+                  const gdn_params_t *p, void *cuda_stream);
+
+/*
+ * gdn_recurrent_step -- one decode token for each of N sequences.
+ *
+ * Walkthrough section 5(2) (torch_recurrent_gated_delta_rule) with one token.
+ * Equal to gdn_chunk_fwd on T = N sequences of length 1 with
+ * final_state = initial_state = state.
+ *
+ *   q, k     [N, Nqk, Dk]   io_dtype
+ *   v        [N, Nv, Dv]    io_dtype
+ *   g, beta  [N, Nv]        fp32
+ *   state    [N, Nv, Dk, Dv] fp32, read and updated IN PLACE
+ *   out      [N, Nv, Dv]    io_dtype; must not overlap any input or the state
+ *   num_seqs N >= 1
+ */
+int gdn_recurrent_step(const void *q, const void *k, const void *v,
+                       const float *g, const float *beta,
+                       float *state, void *out, int32_t num_seqs,
+                       const gdn_params_t *p, void *cuda_stream);
+
+/*
+ * gdn_device_status -- synchronise `cuda_stream`, then read and clear the
+ * library's device-side error word for the current device.  Returns GDN_OK,
+ * GDN_ERR_DEVICE_TIMEOUT if a kernel gave up a bounded wait since the last
+ * call (its outputs are then undefined), or GDN_ERR_CUDA if the stream
+ * reported an error.
+ */
+int gdn_device_status(void *cuda_stream);
+
+/* Human-readable name of a status code (static storage; never NULL). */
+const char *gdn_status_string(int status);
+
+/* ABI version: (major << 16) | minor. */
+int gdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */

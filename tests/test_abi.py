@@ -1,0 +1,113 @@
+"""The C-ABI library: it loads, exports every symbol include/gdn.h declares, and
+rejects bad arguments on the host before any CUDA call (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from gated_deltanet_chunk_b200 import build
+    build.build()
+    import gated_deltanet_chunk_b200 as g
+    return g.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    for n in ("gdn_chunk_fwd", "gdn_recurrent_step", "gdn_status_string", "gdn_device_status",
+              "gdn_version"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    for n in declared_functions():
+        assert hasattr(L, n), n
+
+
+def test_version_and_status_strings(L):
+    assert L.gdn_version() >> 16 == 1
+    for code in range(-7, 1):
+        s = L.gdn_status_string(code).decode()
+        assert s.startswith("GDN")
+    assert "unknown" in L.gdn_status_string(5).decode()
+
+
+# Fake, never-dereferenced, 16-byte aligned addresses: validation must reject
+# these calls on the host before it touches the device or the memory.
+A = 0x100000
+
+
+def _p(**kw):
+    import gated_deltanet_chunk_b200 as g
+    base = dict(nqk=2, nv=4, dk=128, dv=128, io_bf16=True)
+    base.update(kw)
+    return g.make_params(base["nqk"], base["nv"], base["dk"], base["dv"], base["io_bf16"])
+
+
+def _chunk(L, p, q=A, k=A + 0x1000000, v=A + 0x2000000, g=A + 0x3000000, b=A + 0x4000000,
+           s0=None, cu=None, n=2, T=256, C=64, out=A + 0x5000000, sf=None):
+    vp = ctypes.c_void_p
+    return L.gdn_chunk_fwd(vp(q), vp(k), vp(v), vp(g), vp(b), vp(s0), vp(cu), n, T, C, vp(out),
+                           vp(sf), ctypes.byref(p) if p is not None else None, None)
+
+
+def test_validation_rejects_before_launch(L):
+    # NULL params / pointers
+    assert _chunk(L, None) == -1
+    assert _chunk(L, _p(), q=None) == -1
+    assert _chunk(L, _p(), out=None) == -1
+    # shapes
+    assert _chunk(L, _p(nqk=3, nv=4)) == -2            # Nv % Nqk != 0
+    assert _chunk(L, _p(dk=96)) == -2                  # head dim
+    assert _chunk(L, _p(dv=32)) == -2
+    assert _chunk(L, _p(), C=32) == -2                 # chunk size
+    assert _chunk(L, _p(), n=0) == -2                  # no sequences
+    assert _chunk(L, _p(), T=255, n=2) == -2           # uneven split without cu_seqlens
+    assert _chunk(L, _p(), T=-1) == -2
+    # alignment
+    assert _chunk(L, _p(), q=A + 4) == -3
+    assert _chunk(L, _p(), cu=A + 0x6000008) == -3
+    # aliasing: out over v; final_state over q; final_state partially over initial_state
+    assert _chunk(L, _p(), out=A + 0x2000000) == -4
+    assert _chunk(L, _p(), sf=A) == -4
+    assert _chunk(L, _p(), s0=A + 0x7000000, sf=A + 0x7000000 + 4096) == -4
+
+
+def test_recurrent_validation(L):
+    vp = ctypes.c_void_p
+    p = _p()
+    assert L.gdn_recurrent_step(vp(A), vp(A), vp(A), vp(A), vp(A), None, vp(A), 4, ctypes.byref(p), None) == -1
+    assert L.gdn_recurrent_step(vp(A), vp(A + 0x100000), vp(A + 0x200000), vp(A + 0x300000), vp(A + 0x400000),
+                                vp(A + 0x500000), vp(A + 0x500000), 4, ctypes.byref(p), None) == -4
+    assert L.gdn_recurrent_step(vp(A), vp(A + 0x100000), vp(A + 0x200000), vp(A + 0x300000), vp(A + 0x400000),
+                                vp(A + 0x500000), vp(A + 0x900002), 4, ctypes.byref(p), None) == -3
+    bad = _p(nqk=5, nv=4)
+    assert L.gdn_recurrent_step(vp(A), vp(A), vp(A), vp(A), vp(A), vp(A), vp(A), 4, ctypes.byref(bad), None) == -2
+
+
+def test_valid_call_without_gpu_launches_nothing(L):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("only meaningful without a GPU (the fake pointers must never reach a kernel)")
+    rc = _chunk(L, _p())
+    assert rc in (-5, -6)  # the device check fails: no kernel is launched
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    import gated_deltanet_chunk_b200 as g
+    monkeypatch.setattr(g, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(g, "_lib", None)
+    with pytest.raises(ImportError):
+        g.lib()
