@@ -129,9 +129,14 @@ GDN_API int gdn_chunk_fwd(const void* q, const void* k, const void* v, const flo
   a.scale = resolve_scale(p);
   cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
 
-  if (p->kernel == GDN_KERNEL_TC) return GDN_ERR_SHAPE;  // tensor-core kernel: not available for these shapes
-  cudaError_t e = gdn::launch_chunk_simt(a, p->head_k_dim, chunk_size,
-                                         p->io_dtype == GDN_DTYPE_BF16, stream);
+  const int bf16 = p->io_dtype == GDN_DTYPE_BF16;
+  const bool tc_ok = gdn::chunk_tc_supported(p->head_k_dim, p->head_v_dim, chunk_size, bf16, total_tokens);
+  if (p->kernel == GDN_KERNEL_TC && !tc_ok) return GDN_ERR_SHAPE;
+  cudaError_t e;
+  if (tc_ok && p->kernel != GDN_KERNEL_SIMT)
+    e = gdn::launch_chunk_tc(a, total_tokens, stream);
+  else
+    e = gdn::launch_chunk_simt(a, p->head_k_dim, chunk_size, bf16, stream);
   return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
@@ -177,5 +182,7 @@ GDN_API int gdn_recurrent_step(const void* q, const void* k, const void* v, cons
 GDN_API int gdn_device_status(void* cuda_stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(cuda_stream));
   if (e != cudaSuccess) return GDN_ERR_CUDA;
-  return GDN_OK;
+  const unsigned int st = gdn::chunk_tc_take_status();
+  if (st == ~0u) return GDN_ERR_CUDA;
+  return st ? GDN_ERR_DEVICE_TIMEOUT : GDN_OK;
 }

@@ -10,6 +10,12 @@ namespace gdn {
 // fp32 CUDA-core chunked forward; dk in {64,128}, chunk in {64,128}, dv % 32 == 0.
 cudaError_t launch_chunk_simt(const ChunkArgs& a, int dk, int chunk, int io_bf16, cudaStream_t s);
 
+// Tensor-core chunked forward (tcgen05 + TMA): bf16 io, Dk = Dv = 128, chunk 64.
+bool chunk_tc_supported(int dk, int dv, int chunk, int io_bf16, int64_t total_tokens);
+cudaError_t launch_chunk_tc(const ChunkArgs& a, int64_t total_tokens, cudaStream_t s);
+// Reads and clears the tensor-core kernel's device status word (bit 0: a bounded wait expired).
+unsigned int chunk_tc_take_status();
+
 // One-token decode step; dk, dv in {64,128}.
 cudaError_t launch_recurrent_step(const StepArgs& a, int dk, int dv, int io_bf16, cudaStream_t s);
 

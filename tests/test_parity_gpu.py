@@ -94,7 +94,7 @@ def test_split_and_carry_matches_unsplit():
                            w["g"][t:].contiguous(), w["beta"][t:].contiguous(), s1, chunk_size=64)
         torch.cuda.synchronize()
         assert U.rel_inf(U.to_np(torch.cat([o1, o2])), U.to_np(full_o)) < 2e-2
-        assert U.rel_inf(U.to_np(s2), U.to_np(full_s)) < 1e-4
+        assert U.rel_inf(U.to_np(s2), U.to_np(full_s)) < 2e-2
 
 
 def test_in_place_state_and_no_final_state():
@@ -183,3 +183,27 @@ def test_decode_equals_chunk_with_t1():
     torch.cuda.synchronize()
     assert U.rel_inf(U.to_np(o_step), U.to_np(o_chk)) < 1e-5
     assert U.rel_inf(U.to_np(st), U.to_np(s_chk)) < 1e-5
+
+
+# ---------------------------------------------------------------- tensor-core kernel
+@pytest.mark.parametrize("lens,nqk,nv,init", [([64], 1, 1, False), ([1], 1, 1, True), ([65, 63], 1, 2, True),
+                                              ([700, 130, 1], 2, 4, True), ([4096], 4, 8, True)])
+def test_tc_kernel_against_oracle(lens, nqk, nv, init):
+    w = W.make_prefill(lengths=lens, nqk=nqk, nv=nv, d=128, io="bf16", init_state=init, seed=31)
+    _prefill_case(w, 64, kernel="tc", what="tc")
+
+
+def test_tc_kernel_matches_simt_kernel():
+    w = W.make_prefill(num_seqs=3, seq_len=1000, nqk=2, nv=4, d=128, io="bf16", init_state=True, seed=32,
+                       A_hi=0.5)
+    o_tc, s_tc = U.run_gpu_prefill(w, 64, kernel="tc")
+    o_si, s_si = U.run_gpu_prefill(w, 64, kernel="simt")
+    assert U.rel_inf(U.to_np(o_tc), U.to_np(o_si)) < 2e-2
+    assert U.rel_inf(U.to_np(s_tc), U.to_np(s_si)) < 2e-2
+
+
+def test_tc_device_status_clean():
+    import gated_deltanet_chunk_b200 as g
+    w = W.make_prefill(num_seqs=1, seq_len=200, nqk=1, nv=2, d=128, io="bf16", seed=33)
+    U.run_gpu_prefill(w, 64, kernel="tc")
+    assert g.device_status() == 0
