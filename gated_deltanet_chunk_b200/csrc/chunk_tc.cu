@@ -4,10 +4,11 @@
 // v-head, 64-column slice of Dv): the recurrence is separable in the Dv
 // columns.  Two warpgroups run a software pipeline over the sequence's chunks:
 //
-//   intra warpgroup (warps 0-3): everything of chunk c that does not depend on
-//     the state -- gate cumsum, L2 norms, G = [K;Q] K^T, the A and P matrices,
-//     T = (I - A)^-1, U, W -- runs ahead of the serial warpgroup through a ring
-//     of 3 chunk slots in shared memory (plus one TMEM U buffer per slot);
+//   intra warpgroup (warps 0-3): the state-independent part of chunk c -- gate
+//     cumsum, L2 norms, G = [K;Q] K^T, the A and P matrices, T = (I - A)^-1 and
+//     W -- runs ahead of the serial warpgroup.  Raw q/k/v tiles arrive by TMA
+//     in a ring of 3 input slots; the products (W, P, T diag(beta), per-row
+//     scalars) go to a ring of 2 product slots.
 //   serial warpgroup (warps 4-7): the state recurrence, two tensor-core round
 //     trips per chunk.  The fp32 state slice S [128 x 64] lives in registers
 //     (thread d holds row d) and, rounded to bf16, in shared memory as the B
@@ -16,20 +17,20 @@
 // Algebra: the chunkwise form of the "手撕Qwen3-Next" walkthrough, section
 // 一(一)5(1), steps c-f, with the L2 norms folded into row scales
 // (rk = 1/|k|, rq = scale/|q|) so the raw TMA-loaded q/k tiles are the MMA
-// operands.  Gamma[r][i] = exp(gcum_r - gcum_i) for i <= r is formed only below
-// the diagonal (mask before exp), as a product of two factors <= 1 across
-// 16-row blocks.  Per chunk:
+// operands.  Gamma[r][i] = exp(gcum_r - gcum_i) is formed only for i <= r
+// (mask before exp), once per chunk, as the table GK[r][i] = rk_i Gamma[r][i].
 //   G  = [K; Q] K^T                                     tcgen05 M=128 N=64 K=128
-//   A  = -strictLower(diag(beta rk) (K K^T) diag(rk) * Gamma)          CUDA cores
-//   P  = diag(rq) (Q K^T) diag(rk) * Gamma, lower incl. diagonal        CUDA cores
+//   A  = -strictLower(diag(beta rk) (K K^T) * GK)                      CUDA cores
+//   P  = diag(rq) (Q K^T) * GK  (lower incl. diagonal)                  CUDA cores
 //   T  = (I - A)^-1 = R + N^2 R,  R = T_D + N T_D,  N = T_D A_off       3 tcgen05 rounds
 //        (T_D: inverse of A's 16x16 diagonal blocks by forward substitution
-//        in registers; A_off: the strictly block-lower part of A.  N^4 = 0.
+//        in registers; A_off: the strictly block-lower part of A; N^4 = 0.
 //        The 16-row block scheme is the PyPTO README's inverse_pto submodule.)
-//   U  = T diag(beta) V,  W = T diag(beta exp(gcum) rk) K               tcgen05
-//   [Q'S ; W S] = [Q'; W] S,  Q' = diag(exp(gcum) rq) Q                  serial
-//   V' = U - W S;  O = Q'S + P V'                                        serial
-//   S <- exp(g_last) S + K^T diag(rk exp(g_last - gcum)) V'              serial
+//   W  = T diag(beta exp(gcum) rk) K                                    tcgen05
+//   serial:  [KS; QS] = [K; Q] S,  WS = W S,  U = T diag(beta) V        one round
+//            V' = U - W S                                               CUDA cores
+//            PV = P V',  D4 = K^T diag(rk exp(g_last - gcum)) V'        one round
+//            O = diag(exp(gcum) rq) QS + PV;  S <- exp(g_last) S + D4
 // Every accumulation is fp32 in TMEM; MMA operands are bf16.
 //
 // Operand placement: an M=128 A operand is two stacked 64-row tiles; where only
@@ -54,41 +55,45 @@ constexpr int C = 64;
 constexpr int DK = 128;
 constexpr int DVS = 64;        // Dv columns per CTA
 constexpr int kThreads = 256;  // two warpgroups
-constexpr int NS = 3;          // chunk slots in flight
+constexpr int NR = 3;          // raw input slots
+constexpr int NP = 2;          // product slots
 constexpr uint64_t kWaitNs = 1000000000ull;
 
 // ---- shared memory layout (bytes from a 1024-aligned base)
 constexpr int kTile = 64 * 128;  // 64 rows x 128 bytes (64 bf16)
-// one slot: [K_lo | Q_lo | W_lo] [K_hi | Q_hi | W_hi] [V, later P]
-constexpr int SL_KLO = 0, SL_QLO = 1 * kTile, SL_WLO = 2 * kTile;
-constexpr int SL_KHI = 3 * kTile, SL_QHI = 4 * kTile, SL_WHI = 5 * kTile;
-constexpr int SL_VP = 6 * kTile;
-constexpr int kSlot = 7 * kTile;
-constexpr int OFF_X0 = NS * kSlot;       // intra scratch: A_off, N^2, T diag(bw)
-constexpr int OFF_X1 = OFF_X0 + kTile;   // intra scratch: T_D, T diag(beta)
-constexpr int OFF_S = OFF_X1 + kTile;    // serial: S operand, 128 rows (d) x 64 cols
-constexpr int OFF_VP = OFF_S + 2 * kTile;  // serial: V'
-constexpr int OFF_WP = OFF_VP + kTile;     // serial: diag(rk exp(g_last - gcum)) V'
-constexpr int OFF_SCI = OFF_WP + kTile;    // intra scalars
-constexpr int SI_RK = 0, SI_RQ = 64, SI_BETA = 128, SI_GC = 192, SI_EG = 256, SI_BW = 320, SI_F0 = 384,
-              SI_RF = 448, SI_N = 704;  // RF: 4 x 64 table (block 0 unused)
-constexpr int OFF_SCS = OFF_SCI + SI_N * 4;  // per-slot scalars for the serial side
-constexpr int SS_WK = 0, SS_GAMMA = 64, SS_N = 68;
-constexpr int OFF_BAR = OFF_SCS + NS * SS_N * 4;
-// barriers: tma_full[NS], slot_free[NS], intra_full[NS], mma_i, mma_s; then tmem slot, abort flag
-constexpr int BAR_TMA = 0, BAR_FREE = NS, BAR_INTRA = 2 * NS, BAR_MMAI = 3 * NS, BAR_MMAS = 3 * NS + 1;
-constexpr int NBAR = 3 * NS + 2;
+// raw slot: [K_lo | Q_lo] [K_hi | Q_hi] V
+constexpr int RS_KLO = 0, RS_QLO = 1 * kTile, RS_KHI = 2 * kTile, RS_QHI = 3 * kTile, RS_V = 4 * kTile;
+constexpr int kRaw = 5 * kTile;
+// product slot: [W_lo | W_hi | P | T diag(beta)]; W_lo/W_hi hold the GK table
+// while the products are formed and V' / W' once the serial side has read W.
+constexpr int PS_WLO = 0, PS_WHI = 1 * kTile, PS_P = 2 * kTile, PS_TU = 3 * kTile;
+constexpr int kProd = 4 * kTile;
+constexpr int OFF_RAW = 0;
+constexpr int OFF_PROD = NR * kRaw;
+constexpr int OFF_X0 = OFF_PROD + NP * kProd;  // intra scratch: A_off, N^2, T diag(bw)
+constexpr int OFF_X1 = OFF_X0 + kTile;         // intra scratch: T_D
+constexpr int OFF_S = OFF_X1 + kTile;          // serial: S operand, 128 rows (d) x 64 cols
+constexpr int OFF_SCI = OFF_S + 2 * kTile;     // intra scalars
+constexpr int SI_RK = 0, SI_RQ = 64, SI_BETA = 128, SI_GC = 192, SI_BW = 256, SI_N = 320;
+constexpr int OFF_SCP = OFF_SCI + SI_N * 4;    // per-product-slot scalars for the serial side
+constexpr int SP_WK = 0, SP_SQ = 64, SP_GAMMA = 128, SP_N = 132;
+constexpr int OFF_BAR = OFF_SCP + NP * SP_N * 4;
+// barriers: raw_full[NR], raw_free[NR], prod_full[NP], prod_free[NP], mma_i, mma_s
+constexpr int BAR_RAWF = 0, BAR_RAWE = NR, BAR_PRODF = 2 * NR, BAR_PRODE = 2 * NR + NP;
+constexpr int BAR_MMAI = 2 * NR + 2 * NP, BAR_MMAS = BAR_MMAI + 1, NBAR = BAR_MMAS + 1;
 constexpr int SMEM_USED = OFF_BAR + NBAR * 8 + 16;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
 static_assert(OFF_BAR % 8 == 0, "mbarrier alignment");
 static_assert(SMEM_BYTES <= 232448, "shared memory");
 
 // ---- TMEM columns (128 lanes x 512 fp32 columns)
-constexpr uint32_t TM_G = 0;      // G; then N; then N^2 R
-constexpr uint32_t TM_N2 = 64;    // [N^2 | N T_D] (128 cols); then W (128 cols)
-constexpr uint32_t TM_U = 192;    // U of slot s at 192 + 64 s
-constexpr uint32_t TM_D1 = 384;   // serial: [Q'S ; W S], then O
-constexpr uint32_t TM_D4 = 448;   // serial: state update
+constexpr uint32_t TM_G = 0;     // intra: G; then N; then N^2 R
+constexpr uint32_t TM_N2 = 64;   // intra: [N^2 | N T_D] (128 cols); then W (128 cols)
+constexpr uint32_t TM_KQS = 192; // serial: [K S ; Q S]
+constexpr uint32_t TM_WS = 256;  // serial: W S (rows 0..63)
+constexpr uint32_t TM_U = 320;   // serial: U (rows 0..63)
+constexpr uint32_t TM_PV = 384;  // serial: P V' (rows 64..127)
+constexpr uint32_t TM_D4 = 448;  // serial: state update
 constexpr uint32_t TM_COLS = 512;
 
 constexpr uint32_t ID_KK64 = ptx::idesc_bf16_f32(128, 64, false, false);
@@ -108,43 +113,25 @@ __device__ __forceinline__ void mma_k64(uint32_t d, uint32_t a, uint32_t b, uint
     ptx::mma_bf16(d, kdesc(a + 32 * kk), mndesc(b + 2048 * kk, b_lbo), idesc, acc | (kk > 0));
 }
 
+// K = 128 product: A K-major split in two 64-column tiles at a_lo / a_hi, B MN-major at b.
+__device__ __forceinline__ void mma_k128(uint32_t d, uint32_t a_lo, uint32_t a_hi, uint32_t b, uint32_t b_lbo,
+                                         uint32_t idesc) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk)
+    ptx::mma_bf16(d, kdesc((kk < 4 ? a_lo : a_hi) + 32 * (kk & 3)), mndesc(b + 2048 * kk, b_lbo), idesc, kk > 0);
+}
+
 __device__ __forceinline__ void tmem_row64(uint32_t taddr, float* v) {
   ptx::tmem_ld32(taddr, v);
   ptx::tmem_ld32(taddr + 32, v + 32);
   ptx::tmem_ld_wait();
 }
 
-// row[i] <- row[i] * f * rk_i * Gamma[r][i] for i < r (i <= r when incl_diag), else 0,
-// with Gamma[r][i] = exp(gcum_r - gcum_i).  Columns left of r's 16-row block use
-// the table RF[b][i] = rk_i exp(gcum_{16b} - gcum_i) times exp(gcum_r - gcum_{16b});
-// only the 16 columns of r's own block take a direct exp.  Branch-free: every
-// choice is a select on compile-time column indices.
-__device__ __forceinline__ void scale_gamma_row(float* row, const float* si, int r, float f, bool incl_diag) {
-  const int b = r >> 4, li = r & 15;
-  const float gr = si[SI_GC + r];
-  const float fb = f * si[SI_F0 + r];
-  const float* rf = si + SI_RF + 64 * b;
-  const float* gb = si + SI_GC + 16 * b;
-  const float* kb = si + SI_RK + 16 * b;
-  float own[16];
-#pragma unroll
-  for (int jj = 0; jj < 16; ++jj) {
-    const bool on = incl_diag ? (jj <= li) : (jj < li);
-    own[jj] = on ? f * kb[jj] * fast_exp(fminf(gr - gb[jj], 0.f)) : 0.f;
-  }
-#pragma unroll
-  for (int cb = 0; cb < 4; ++cb)
-#pragma unroll
-    for (int jj = 0; jj < 16; ++jj) {
-      const int i = 16 * cb + jj;
-      const float fac = (cb < b) ? fb * rf[i] : ((cb == b) ? own[jj] : 0.f);
-      row[i] *= fac;
-    }
-}
+__device__ __forceinline__ void named_bar(int id) { asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory"); }
 
-__device__ __forceinline__ void named_bar(int id) {
-  asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory");
-}
+// GK table: fp32 [64][64], rows of 256 bytes with the 16-byte chunk k of row r
+// stored at chunk position k ^ (r & 7) (conflict-free row reads).
+__device__ __forceinline__ int gk_index(int r, int i) { return r * 64 + ((((i >> 2) ^ (r & 7))) << 2) + (i & 3); }
 
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -163,17 +150,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_BAR + NBAR * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_BAR + NBAR * 8 + 4);
   float* si = reinterpret_cast<float*>(sm + OFF_SCI);
-  float* ss = reinterpret_cast<float*>(sm + OFF_SCS);
+  float* sp = reinterpret_cast<float*>(sm + OFF_SCP);
 
   int64_t seq_start, seq_end;
   seq_bounds(a.cu, a.uniform_len, n, seq_start, seq_end);
   const int nchunks = (int)((seq_end - seq_start + C - 1) / C);
 
   if (tid == 0) {
-    for (int i = 0; i < NS; ++i) {
-      ptx::mbar_init(bars + BAR_TMA + i, 1);
-      ptx::mbar_init(bars + BAR_FREE + i, 1);
-      ptx::mbar_init(bars + BAR_INTRA + i, 1);
+    for (int i = 0; i < NR; ++i) {
+      ptx::mbar_init(bars + BAR_RAWF + i, 1);
+      ptx::mbar_init(bars + BAR_RAWE + i, 1);
+    }
+    for (int i = 0; i < NP; ++i) {
+      ptx::mbar_init(bars + BAR_PRODF + i, 1);
+      ptx::mbar_init(bars + BAR_PRODE + i, 1);
     }
     ptx::mbar_init(bars + BAR_MMAI, 1);
     ptx::mbar_init(bars + BAR_MMAS, 1);
@@ -200,16 +190,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     // =====================================================================
     const int t = tid;  // 0..127
     auto issue_tma = [&](int chunk) {
-      const int s = chunk % NS;
+      const int s = chunk % NR;
       const int t0 = (int)(seq_start + (int64_t)chunk * C);
-      uint8_t* sl = sm + s * kSlot;
-      uint64_t* bar = bars + BAR_TMA + s;
+      uint8_t* rs = sm + OFF_RAW + s * kRaw;
+      uint64_t* bar = bars + BAR_RAWF + s;
       ptx::mbar_arrive_expect_tx(bar, 5 * kTile);
-      ptx::tma_load_3d(sl + SL_KLO, &tm_k, bar, 0, j, t0);
-      ptx::tma_load_3d(sl + SL_KHI, &tm_k, bar, 64, j, t0);
-      ptx::tma_load_3d(sl + SL_QLO, &tm_q, bar, 0, j, t0);
-      ptx::tma_load_3d(sl + SL_QHI, &tm_q, bar, 64, j, t0);
-      ptx::tma_load_3d(sl + SL_VP, &tm_v, bar, slice * DVS, h, t0);
+      ptx::tma_load_3d(rs + RS_KLO, &tm_k, bar, 0, j, t0);
+      ptx::tma_load_3d(rs + RS_KHI, &tm_k, bar, 64, j, t0);
+      ptx::tma_load_3d(rs + RS_QLO, &tm_q, bar, 0, j, t0);
+      ptx::tma_load_3d(rs + RS_QHI, &tm_q, bar, 64, j, t0);
+      ptx::tma_load_3d(rs + RS_V, &tm_v, bar, slice * DVS, h, t0);
     };
     uint32_t ph_mma = 0;
     bool ok = true;
@@ -229,8 +219,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::tc_fence_before();
       named_bar(1);
     };
+    // The raw slot of chunk c' becomes free when the serial side has finished chunk c' - NR.
+    auto prefetch = [&](int cn) {
+      if (cn >= nchunks) return;
+      if (cn >= NR && !ptx::mbar_wait_bounded(bars + BAR_RAWE + cn % NR, (uint32_t)((cn / NR - 1) & 1), kWaitNs))
+        *abort_flag = 1;
+      issue_tma(cn);
+    };
 
-    if (t == 0 && nchunks > 0) issue_tma(0);
+    if (t == 96) {  // warp 3 issues the tensor loads
+      prefetch(0);
+      prefetch(1);
+    }
     float g_next = 0.f, b_next = 0.f;
     if (t < 64 && seq_start + t < seq_end) {
       g_next = a.g[(size_t)(seq_start + t) * nv + h];
@@ -238,20 +238,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     for (int c = 0; c < nchunks && ok; ++c) {
-      const int s = c % NS;
+      const int rsl = c % NR, psl = c % NP;
       const int64_t c0 = seq_start + (int64_t)c * C;
-      uint8_t* sl = sm + s * kSlot;
-      const uint32_t sa = sb + s * kSlot;
-      float* sss = ss + s * SS_N;
+      uint8_t* rs = sm + OFF_RAW + rsl * kRaw;
+      const uint32_t ra = sb + OFF_RAW + rsl * kRaw;
+      uint8_t* ps = sm + OFF_PROD + psl * kProd;
+      const uint32_t pa = sb + OFF_PROD + psl * kProd;
+      float* spp = sp + psl * SP_N;
+      float* gk = reinterpret_cast<float*>(ps + PS_WLO);  // 16 KB: the W_lo / W_hi tiles
 
-      // (a) prefetch the next chunk's tiles once its slot is free
-      if (t == 0 && c + 1 < nchunks) {
-        const int cn = c + 1;
-        if (cn >= NS && !ptx::mbar_wait_bounded(bars + BAR_FREE + cn % NS, (uint32_t)((cn / NS - 1) & 1), kWaitNs))
-          *abort_flag = 1;
-        issue_tma(cn);
-      }
-      // (b) gates: beta and the warp-local cumsum of g; prefetch the next chunk's gates
+      // gates: beta and the warp-local cumsum of g; prefetch the next chunk's gates
       if (t < 64) {
         float gv = g_next;
         si[SI_BETA + t] = b_next;
@@ -269,24 +265,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           b_next = a.beta[(size_t)tn * nv + h];
         }
       }
-      // (c) tiles of this chunk
-      wait_bar(bars + BAR_TMA + s, (uint32_t)((c / NS) & 1));
+      // the product slot must have been released by the serial side (chunk c - NP)
+      if (t == 0 && c >= NP &&
+          !ptx::mbar_wait_bounded(bars + BAR_PRODE + psl, (uint32_t)((c / NP - 1) & 1), kWaitNs))
+        *abort_flag = 1;
+      wait_bar(bars + BAR_RAWF + rsl, (uint32_t)((c / NR) & 1));
       if (!ok) break;
-      // (d) G = [K; Q] K^T
+      // G = [K; Q] K^T
       if (t == 0) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t ao = (kk < 4 ? SL_KLO : SL_KHI) + (kk & 3) * 32;
-          ptx::mma_bf16(tmem + TM_G, kdesc(sa + ao), kdesc(sa + ao), ID_KK64, kk > 0);
+          const uint32_t ao = (kk < 4 ? RS_KLO : RS_KHI) + (kk & 3) * 32;
+          ptx::mma_bf16(tmem + TM_G, kdesc(ra + ao), kdesc(ra + ao), ID_KK64, kk > 0);
         }
         ptx::mma_commit(bars + BAR_MMAI);
       }
-      // (e) norms: threads 0..63 keys (rk), 64..127 queries (rq); cumsum fix-up
       if (t >= 32 && t < 64) si[SI_GC + t] += si[SI_GC + 31];
+      // norms: threads 0..63 keys (rk), 64..127 queries (rq)
       {
         const int r = t & 63;
-        const uint8_t* lo = sl + (t < 64 ? SL_KLO : SL_QLO);
-        const uint8_t* hi = sl + (t < 64 ? SL_KHI : SL_QHI);
+        const uint8_t* lo = rs + (t < 64 ? RS_KLO : RS_QLO);
+        const uint8_t* hi = rs + (t < 64 ? RS_KHI : RS_QHI);
         float v[64];
         float sq = 0.f;
         ptx::ld_row_bf16(lo, r, v);
@@ -301,80 +300,72 @@ __global__ void __launch_bounds__(kThreads, 1)
         si[(t < 64 ? SI_RK : SI_RQ) + r] = valid ? f : 0.f;
       }
       named_bar(1);
-      // (f) derived per-row scalars and the cross-block decay table
+      // GK[r][i] = rk_i exp(gcum_r - gcum_i) for i <= r (else 0); row scalars
+#pragma unroll 4
+      for (int e = t; e < 64 * 64; e += 128) {
+        const int r = e >> 6, i = e & 63;
+        const float val = (i <= r) ? si[SI_RK + i] * fast_exp(si[SI_GC + r] - si[SI_GC + i]) : 0.f;
+        gk[gk_index(r, i)] = val;
+      }
       if (t < 64) {
         const float gl = si[SI_GC + 63], gr = si[SI_GC + t];
         const float eg = fast_exp(gr);
         const float rk = si[SI_RK + t];
-        si[SI_EG + t] = eg;
         si[SI_BW + t] = si[SI_BETA + t] * eg * rk;
-        si[SI_F0 + t] = fast_exp(gr - si[SI_GC + (t & ~15)]);  // exp(gcum_r - gcum_{block start})
-        sss[SS_WK + t] = rk * fast_exp(gl - gr);
-        if (t == 0) sss[SS_GAMMA] = fast_exp(gl);
-      } else {
-        // RF[b][i] = rk_i exp(gcum_{16b} - gcum_i) for i < 16 b, b = 1..3 (rows of block >= b)
-        for (int e = t - 64; e < 256; e += 64) {
-          const int b = e >> 6, i = e & 63;
-          float val = 0.f;
-          if (b >= 1 && i < 16 * b) val = si[SI_RK + i] * fast_exp(si[SI_GC + 16 * b] - si[SI_GC + i]);
-          si[SI_RF + e] = val;
-        }
+        spp[SP_WK + t] = rk * fast_exp(gl - gr);
+        spp[SP_SQ + t] = eg * si[SI_RQ + t];
+        if (t == 0) spp[SP_GAMMA] = fast_exp(gl);
       }
-      // (g) G ready
-      wait_mma();
+      wait_mma();  // G ready (the named barrier inside also publishes GK)
       if (!ok) break;
-      // (h) A rows + diagonal-block inverse (threads 0..63); P rows + Q' in place (threads 64..127)
-      // keep[]: query-row threads hold their P row until V has been consumed;
-      //         key-row threads hold R = T_D + N T_D for T = R + N^2 R.
-      float keep[64];
+      // A rows + diagonal-block inverse (threads 0..63); P rows (threads 64..127)
+      float keep[64];  // key-row threads: R = T_D + N T_D, kept for T = R + N^2 R
       float t16[16];   // key-row threads: strictly lower part of this row's T_D block
-      if (t < 64) {
-        const int r = t, b = r >> 4, li = lane & 15;
+      {
+        const int r = t & 63;
         float av[64];
         tmem_row64(tl + TM_G, av);
-        const float fr = -si[SI_BETA + r] * si[SI_RK + r];
-        scale_gamma_row(av, si, r, fr, false);
+        const float f = (t < 64) ? -si[SI_BETA + r] * si[SI_RK + r] : si[SI_RQ + r];
+        const float4* gkr = reinterpret_cast<const float4*>(gk + r * 64);
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj)
-          t16[jj] = (warp == 0) ? (lane < 16 ? av[jj] : av[16 + jj]) : (lane < 16 ? av[32 + jj] : av[48 + jj]);
+        for (int k4 = 0; k4 < 16; ++k4) {
+          const float4 x = gkr[k4 ^ (r & 7)];
+          av[4 * k4 + 0] *= f * x.x;
+          av[4 * k4 + 1] *= f * x.y;
+          av[4 * k4 + 2] *= f * x.z;
+          av[4 * k4 + 3] *= f * x.w;
+        }
+        if (t < 64) {
+          const int b = r >> 4, li = lane & 15;
 #pragma unroll
-        for (int m = 1; m < 15; ++m) {
-          const float coef = t16[m];
+          for (int i = 0; i < 64; ++i) av[i] = (i == r) ? 0.f : av[i];  // strictly lower
 #pragma unroll
-          for (int jj = 0; jj < m; ++jj) {
-            const float bj = __shfl_sync(0xffffffffu, t16[jj], (lane & 16) | m);
-            if (li > m) t16[jj] = fmaf(coef, bj, t16[jj]);
+          for (int jj = 0; jj < 16; ++jj)
+            t16[jj] = (warp == 0) ? (lane < 16 ? av[jj] : av[16 + jj]) : (lane < 16 ? av[32 + jj] : av[48 + jj]);
+#pragma unroll
+          for (int m = 1; m < 15; ++m) {
+            const float coef = t16[m];
+#pragma unroll
+            for (int jj = 0; jj < m; ++jj) {
+              const float bj = __shfl_sync(0xffffffffu, t16[jj], (lane & 16) | m);
+              if (li > m) t16[jj] = fmaf(coef, bj, t16[jj]);
+            }
           }
-        }
-        float td[64];
 #pragma unroll
-        for (int cc = 0; cc < 64; ++cc) {
-          const int cb = cc >> 4, cj = cc & 15;
-          td[cc] = (cb == b) ? (cj < li ? t16[cj] : (cj == li ? 1.f : 0.f)) : 0.f;
-        }
-        ptx::st_row_bf16(sm + OFF_X1, r, td);
+          for (int cc = 0; cc < 64; ++cc) {
+            const int cb = cc >> 4, cj = cc & 15;
+            keep[cc] = (cb == b) ? (cj < li ? t16[cj] : (cj == li ? 1.f : 0.f)) : 0.f;
+          }
+          ptx::st_row_bf16(sm + OFF_X1, r, keep);  // T_D
 #pragma unroll
-        for (int cc = 0; cc < 64; ++cc) av[cc] = (cc < 16 * b) ? av[cc] : 0.f;
-        ptx::st_row_bf16(sm + OFF_X0, r, av);
-      } else {
-        const int r = t - 64, b = r >> 4;
-        float* prow = keep;
-        tmem_row64(tl + TM_G, prow);
-        const float fr = si[SI_RQ + r];
-        scale_gamma_row(prow, si, r, fr, true);
-        const float qf = si[SI_EG + r] * fr;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint8_t* qt = sl + (half ? SL_QHI : SL_QLO);
-          float qv[64];
-          ptx::ld_row_bf16(qt, r, qv);
-#pragma unroll
-          for (int e = 0; e < 64; ++e) qv[e] *= qf;
-          ptx::st_row_bf16(qt, r, qv);
+          for (int cc = 0; cc < 64; ++cc) av[cc] = (cc < 16 * b) ? av[cc] : 0.f;
+          ptx::st_row_bf16(sm + OFF_X0, r, av);  // A_off
+        } else {
+          ptx::st_row_bf16(ps + PS_P, r, av);  // P
         }
       }
       publish();
-      // (i) N = T_D A_off   (A = [T_D; junk]: rows land in lanes 0..63)
+      // N = T_D A_off   (A = [T_D; junk]: rows land in lanes 0..63)
       if (t == 0) {
         ptx::tc_fence_after();
         mma_k64(tmem + TM_G, sb + OFF_X1, sb + OFF_X0, 8192, ID_KMN64, 0);
@@ -385,13 +376,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (t < 64) {
         float x[64];
         tmem_row64(tl + TM_G, x);
-        ptx::st_row_bf16(sl + SL_WLO, t, x);  // N (the W slot is free until W is formed)
+        ptx::st_row_bf16(ps + PS_WLO, t, x);  // N (the GK table has been consumed)
       }
       publish();
-      // (j) [N^2 | N T_D] = N [N | T_D]
+      // [N^2 | N T_D] = N [N | T_D]
       if (t == 0) {
         ptx::tc_fence_after();
-        mma_k64(tmem + TM_N2, sa + SL_WLO, sa + SL_WLO, (uint32_t)(OFF_X1 - (s * kSlot + SL_WLO)), ID_KMN128, 0);
+        mma_k64(tmem + TM_N2, pa + PS_WLO, pa + PS_WLO, (uint32_t)(OFF_X1 - (OFF_PROD + psl * kProd + PS_WLO)),
+                ID_KMN128, 0);
         ptx::mma_commit(bars + BAR_MMAI);
       }
       wait_mma();
@@ -408,13 +400,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float tdv = (cb == b) ? (cj < li ? t16[cj] : (cj == li ? 1.f : 0.f)) : 0.f;
           keep[cc] = tdv + x[cc];  // R = T_D + N T_D
         }
-        ptx::st_row_bf16(sl + SL_WHI, r, keep);
+        ptx::st_row_bf16(ps + PS_WHI, r, keep);
       }
       publish();
-      // (k) N^2 R
+      // N^2 R
       if (t == 0) {
         ptx::tc_fence_after();
-        mma_k64(tmem + TM_G, sb + OFF_X0, sa + SL_WHI, 8192, ID_KMN64, 0);
+        mma_k64(tmem + TM_G, sb + OFF_X0, pa + PS_WHI, 8192, ID_KMN64, 0);
         ptx::mma_commit(bars + BAR_MMAI);
       }
       wait_mma();
@@ -429,14 +421,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::st_row_bf16(sm + OFF_X0, t, keep);  // T diag(beta exp(gcum) rk)
 #pragma unroll
         for (int cc = 0; cc < 64; ++cc) keep[cc] = x[cc] * si[SI_BETA + cc];
-        ptx::st_row_bf16(sm + OFF_X1, t, keep);  // T diag(beta)
+        ptx::st_row_bf16(ps + PS_TU, t, keep);  // T diag(beta), for U on the serial side
       }
       publish();
-      // (l) W = T diag(bw) K (rows 0..63), U = T diag(beta) V (rows 64..127 of U[s])
+      // W = T diag(bw) K   (A = [T diag(bw); junk])
       if (t == 0) {
         ptx::tc_fence_after();
-        mma_k64(tmem + TM_U + 64 * s, sb + OFF_X0, sa + SL_VP, 8192, ID_KMN64, 0);
-        mma_k64(tmem + TM_N2, sb + OFF_X0, sa + SL_KLO, SL_KHI - SL_KLO, ID_KMN128, 0);
+        mma_k64(tmem + TM_N2, sb + OFF_X0, ra + RS_KLO, RS_KHI - RS_KLO, ID_KMN128, 0);
         ptx::mma_commit(bars + BAR_MMAI);
       }
       wait_mma();
@@ -444,14 +435,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (t < 64) {
         float x[64];
         tmem_row64(tl + TM_N2, x);
-        ptx::st_row_bf16(sl + SL_WLO, t, x);
+        ptx::st_row_bf16(ps + PS_WLO, t, x);
         tmem_row64(tl + TM_N2 + 64, x);
-        ptx::st_row_bf16(sl + SL_WHI, t, x);
-      } else {
-        ptx::st_row_bf16(sl + SL_VP, t - 64, keep);  // P row; V has been consumed by U
+        ptx::st_row_bf16(ps + PS_WHI, t, x);
       }
       publish();
-      if (t == 0) ptx::mbar_arrive(bars + BAR_INTRA + s);
+      if (t == 0) ptx::mbar_arrive(bars + BAR_PRODF + psl);
+      // tiles of chunk c + 2: their slot was used by chunk c - 1, which the
+      // serial side has finished by now (it only lags this side by one chunk)
+      if (t == 96) prefetch(c + 2);
     }
     if (!ok && t == 0) atomicOr(&g_status, 1u);
   } else {
@@ -494,72 +486,80 @@ __global__ void __launch_bounds__(kThreads, 1)
       named_bar(2);
     };
 
+    float opart[64];  // lanes 64..127: diag(exp(gcum) rq) Q S
     for (int c = 0; c < nchunks && ok; ++c) {
-      const int s = c % NS;
+      const int rsl = c % NR, psl = c % NP;
       const int64_t c0 = seq_start + (int64_t)c * C;
-      const uint32_t sa = sb + s * kSlot;
-      const float* sss = ss + s * SS_N;
-      wait_bar(bars + BAR_INTRA + s, (uint32_t)((c / NS) & 1));
+      const uint32_t ra = sb + OFF_RAW + rsl * kRaw;
+      uint8_t* ps = sm + OFF_PROD + psl * kProd;
+      const uint32_t pa = sb + OFF_PROD + psl * kProd;
+      const float* spp = sp + psl * SP_N;
+      wait_bar(bars + BAR_PRODF + psl, (uint32_t)((c / NP) & 1));
       if (!ok) break;
-      // [Q'; W] S: rows 0..63 Q'S, rows 64..127 W S
+      // [K S; Q S],  W S (A = [W; junk]),  U = T diag(beta) V (A = [Tb; junk])
       if (t == 0) {
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t ao = (kk < 4 ? SL_QLO : SL_QHI) + (kk & 3) * 32;
-          ptx::mma_bf16(tmem + TM_D1, kdesc(sa + ao), mndesc(sb + OFF_S + 2048 * kk, 8192), ID_KMN64, kk > 0);
-        }
+        mma_k128(tmem + TM_KQS, ra + RS_KLO, ra + RS_KHI, sb + OFF_S, 8192, ID_KMN64);
+        mma_k128(tmem + TM_WS, pa + PS_WLO, pa + PS_WHI, sb + OFF_S, 8192, ID_KMN64);
+        mma_k64(tmem + TM_U, pa + PS_TU, ra + RS_V, 8192, ID_KMN64, 0);
         ptx::mma_commit(bars + BAR_MMAS);
       }
       wait_mma();
       if (!ok) break;
-      // V' = U - W S and diag(rk exp(g_last - gcum)) V'  (lanes 64..127)
-      if (t >= 64) {
-        const int r = t - 64;
+      if (t < 64) {
+        // V' = U - W S, and W' = diag(rk exp(g_last - gcum)) V'  (into the W tiles)
         float u[64], ws[64];
-        tmem_row64(tl + TM_U + 64 * s, u);
-        tmem_row64(tl + TM_D1, ws);
+        tmem_row64(tl + TM_U, u);
+        tmem_row64(tl + TM_WS, ws);
 #pragma unroll
         for (int cc = 0; cc < 64; ++cc) u[cc] -= ws[cc];
-        ptx::st_row_bf16(sm + OFF_VP, r, u);
-        const float w = sss[SS_WK + r];
+        ptx::st_row_bf16(ps + PS_WLO, t, u);
+        const float w = spp[SP_WK + t];
 #pragma unroll
         for (int cc = 0; cc < 64; ++cc) u[cc] *= w;
-        ptx::st_row_bf16(sm + OFF_WP, r, u);
+        ptx::st_row_bf16(ps + PS_WHI, t, u);
+      } else {
+        // Q S scaled by exp(gcum) rq, kept for the output
+        tmem_row64(tl + TM_KQS, opart);
+        const float f = spp[SP_SQ + t - 64];
+#pragma unroll
+        for (int cc = 0; cc < 64; ++cc) opart[cc] *= f;
       }
       publish();
-      // O: D1[0..63] += P V' (A = [P; junk]);  D4 = K^T W'
+      // P V' (A = [junk; P]: rows land in lanes 64..127) and D4 = K^T W'
       if (t == 0) {
         ptx::tc_fence_after();
-        mma_k64(tmem + TM_D1, sa + SL_VP, sb + OFF_VP, 8192, ID_KMN64, 1);
+        mma_k64(tmem + TM_PV, pa + PS_P - kTile, pa + PS_WLO, 8192, ID_KMN64, 0);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          ptx::mma_bf16(tmem + TM_D4, mndesc(sa + SL_KLO + 2048 * kk, SL_KHI - SL_KLO),
-                        mndesc(sb + OFF_WP + 2048 * kk, 8192), ID_MNMN64, kk > 0);
+          ptx::mma_bf16(tmem + TM_D4, mndesc(ra + RS_KLO + 2048 * kk, RS_KHI - RS_KLO),
+                        mndesc(pa + PS_WHI + 2048 * kk, 8192), ID_MNMN64, kk > 0);
         ptx::mma_commit(bars + BAR_MMAS);
       }
       wait_mma();
       if (!ok) break;
-      // outputs (lanes 0..63) and the state update (all lanes)
-      if (t < 64) {
-        const int64_t tok = c0 + t;
+      if (t >= 64) {
+        const int r = t - 64;
+        const int64_t tok = c0 + r;
         float o[64];
-        tmem_row64(tl + TM_D1, o);
+        tmem_row64(tl + TM_PV, o);
         if (tok < seq_end) {
           uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + ((size_t)tok * nv + h) * dv +
                                                  slice * DVS);
 #pragma unroll
           for (int cc = 0; cc < 8; ++cc) {
+            const float* x = o + 8 * cc;
+            const float* y = opart + 8 * cc;
             uint4 w;
-            w.x = ptx::pack_bf16x2(o[8 * cc + 0], o[8 * cc + 1]);
-            w.y = ptx::pack_bf16x2(o[8 * cc + 2], o[8 * cc + 3]);
-            w.z = ptx::pack_bf16x2(o[8 * cc + 4], o[8 * cc + 5]);
-            w.w = ptx::pack_bf16x2(o[8 * cc + 6], o[8 * cc + 7]);
+            w.x = ptx::pack_bf16x2(x[0] + y[0], x[1] + y[1]);
+            w.y = ptx::pack_bf16x2(x[2] + y[2], x[3] + y[3]);
+            w.z = ptx::pack_bf16x2(x[4] + y[4], x[5] + y[5]);
+            w.w = ptx::pack_bf16x2(x[6] + y[6], x[7] + y[7]);
             orow[cc] = w;
           }
         }
       }
       {
-        const float decay = sss[SS_GAMMA];
+        const float decay = spp[SP_GAMMA];
         float x[64];
         tmem_row64(tl + TM_D4, x);
 #pragma unroll
@@ -567,7 +567,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::st_row_bf16(sm + OFF_S, t, S);
       }
       publish();
-      if (t == 0) ptx::mbar_arrive(bars + BAR_FREE + s);
+      if (t == 0) {
+        ptx::mbar_arrive(bars + BAR_PRODE + psl);
+        ptx::mbar_arrive(bars + BAR_RAWE + rsl);
+      }
     }
     if (ok && a.s_final) {
       float4* dst = reinterpret_cast<float4*>(a.s_final + st_off);
