@@ -172,8 +172,12 @@ def run_ours(args, world, rank, local):
 
     dev = torch.device("cuda", local)
     peaks, peak_src = load_peaks()
+    if args.no_prefill:  # profiling helper: the decode workload alone
+        stream = torch.cuda.current_stream(dev)
+        return {"metric": METRIC, "decode": run_decode(args, world, rank, dev, stream, peaks, peak_src)}
     wl = W.WORKLOADS[PREFILL]
-    host = W.make_workload(PREFILL, seed=2 + rank)          # each rank: its own sequences
+    over = {"seq_len": args.seq_len} if args.seq_len else {}
+    host = W.make_workload(PREFILL, seed=2 + rank, **over)  # each rank: its own sequences
     n, T, nqk, nv, D, C = wl.num_seqs, host["T"], wl.nqk, wl.nv, wl.d, wl.chunk
     d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in host.items()}
     out = torch.empty(T, nv, D, dtype=torch.bfloat16, device=dev)
@@ -217,7 +221,7 @@ def run_ours(args, world, rank, local):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f32", "data": "synthetic (seeded; workloads/)",
+        "dtype": "bf16", "data": "synthetic (seeded; workloads/)",
         "config": {"workload": PREFILL, "num_seqs": n, "seq_len": T // n, "nqk": nqk, "nv": nv,
                    "dk": D, "dv": D, "chunk": C, "io": "bf16", "state": "fp32",
                    "initial_state": "zeros", "l2": "inputs 1.63 GB > 126 MB L2; no flush",
@@ -284,7 +288,7 @@ def run_decode(args, world, rank, dev, stream, peaks, peak_src):
     import gated_deltanet_chunk_b200 as gdn
     import workloads as W
     wl = W.WORKLOADS[DECODE]
-    steps = wl.steps
+    steps = args.decode_steps or wl.steps
     d = W.make_decode(num_seqs=wl.num_seqs, steps=steps, nqk=wl.nqk, nv=wl.nv, d=wl.d, io=wl.io,
                       seed=4 + rank, device=str(dev))
     state = d["initial_state"]
@@ -351,6 +355,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true", help="time only the decode workload")
+    ap.add_argument("--seq-len", type=int, default=0,
+                    help="override the prefill sequence length (profiling of smaller cases)")
+    ap.add_argument("--decode-steps", type=int, default=0,
+                    help="override the number of decode steps (profiling of smaller cases)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=4096)

@@ -54,7 +54,7 @@ __device__ unsigned int g_status;  // bit 0: a bounded wait expired
 constexpr int C = 64;
 constexpr int DK = 128;
 constexpr int DVS = 64;        // Dv columns per CTA
-constexpr int kThreads = 256;  // two warpgroups
+constexpr int kThreads = 384;  // 8 intra warps + 4 serial warps
 constexpr int NR = 3;          // raw input slots
 constexpr int NP = 2;          // product slots
 constexpr uint64_t kWaitNs = 1000000000ull;
@@ -74,7 +74,7 @@ constexpr int OFF_X0 = OFF_PROD + NP * kProd;  // intra scratch: A_off, N^2, T d
 constexpr int OFF_X1 = OFF_X0 + kTile;         // intra scratch: T_D
 constexpr int OFF_S = OFF_X1 + kTile;          // serial: S operand, 128 rows (d) x 64 cols
 constexpr int OFF_SCI = OFF_S + 2 * kTile;     // intra scalars
-constexpr int SI_RK = 0, SI_RQ = 64, SI_BETA = 128, SI_GC = 192, SI_BW = 256, SI_N = 320;
+constexpr int SI_RK = 0, SI_RQ = 64, SI_BETA = 128, SI_GC = 192, SI_BW = 256, SI_NP = 320, SI_N = 576;
 constexpr int OFF_SCP = OFF_SCI + SI_N * 4;    // per-product-slot scalars for the serial side
 constexpr int SP_WK = 0, SP_SQ = 64, SP_GAMMA = 128, SP_N = 132;
 constexpr int OFF_BAR = OFF_SCP + NP * SP_N * 4;
@@ -127,7 +127,9 @@ __device__ __forceinline__ void tmem_row64(uint32_t taddr, float* v) {
   ptx::tmem_ld_wait();
 }
 
-__device__ __forceinline__ void named_bar(int id) { asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory"); }
+__device__ __forceinline__ void named_bar_n(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
 
 // GK table: fp32 [64][64], rows of 256 bytes with the 16-byte chunk k of row r
 // stored at chunk position k ^ (r & 7) (conflict-free row reads).
@@ -184,11 +186,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);  // this warp's TMEM lane quarter
   const uint32_t sb = ptx::smem_u32(sm);
 
-  if (warp < 4) {
+  if (warp < 8) {
     // =====================================================================
-    // intra warpgroup
+    // intra warps (0-7): thread (quarter q = warp % 4, half h = warp / 4, lane)
+    // owns columns [32h, 32h + 32) of accumulator row 32q + lane.
     // =====================================================================
-    const int t = tid;  // 0..127
+    const int t = tid;  // 0..255
+    const int q = warp & 3, hf = warp >> 2;
+    const int row = 32 * q + lane;  // accumulator row: 0..63 keys, 64..127 queries
+    const int r = row & 63;
+    const int c0 = 32 * hf;
+    const bool krow = q < 2;
+    // the 16x16 diagonal block of key row r lies in this thread's half
+    const bool diag_here = krow && ((r >> 5) == hf);
+    const int li = lane & 15;
     auto issue_tma = [&](int chunk) {
       const int s = chunk % NR;
       const int t0 = (int)(seq_start + (int64_t)chunk * C);
@@ -206,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // One thread polls the mbarrier; the others park at the named barrier.
     auto wait_bar = [&](uint64_t* bar, uint32_t parity) {
       if (t == 0 && !ptx::mbar_wait_bounded(bar, parity, kWaitNs)) *abort_flag = 1;
-      named_bar(1);
+      named_bar_n(1, 256);
       ok = (*abort_flag == 0);
       ptx::tc_fence_after();
     };
@@ -217,7 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto publish = [&]() {
       ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
-      named_bar(1);
+      named_bar_n(1, 256);
     };
     // The raw slot of chunk c' becomes free when the serial side has finished chunk c' - NR.
     auto prefetch = [&](int cn) {
@@ -226,8 +237,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 1;
       issue_tma(cn);
     };
+    // this thread's 32 columns of T_D (block-diagonal inverse) for key row r
+    auto td_half = [&](const float* t16, float* out32) {
+#pragma unroll
+      for (int cc = 0; cc < 32; ++cc) {
+        const int cj = cc & 15;
+        const bool same_block = (cc >> 4) == (lane >> 4);
+        out32[cc] = (diag_here && same_block) ? (cj < li ? t16[cj] : (cj == li ? 1.f : 0.f)) : 0.f;
+      }
+    };
 
-    if (t == 96) {  // warp 3 issues the tensor loads
+    if (t == 224) {  // a query-row warp issues the tensor loads
       prefetch(0);
       prefetch(1);
     }
@@ -239,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     for (int c = 0; c < nchunks && ok; ++c) {
       const int rsl = c % NR, psl = c % NP;
-      const int64_t c0 = seq_start + (int64_t)c * C;
+      const int64_t c0t = seq_start + (int64_t)c * C;
       uint8_t* rs = sm + OFF_RAW + rsl * kRaw;
       const uint32_t ra = sb + OFF_RAW + rsl * kRaw;
       uint8_t* ps = sm + OFF_PROD + psl * kProd;
@@ -257,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane >= o) gv += y;
         }
         si[SI_GC + t] = gv;
-        const int64_t tn = c0 + C + t;
+        const int64_t tn = c0t + C + t;
         g_next = 0.f;
         b_next = 0.f;
         if (tn < seq_end) {
@@ -281,31 +301,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::mma_commit(bars + BAR_MMAI);
       }
       if (t >= 32 && t < 64) si[SI_GC + t] += si[SI_GC + 31];
-      // norms: threads 0..63 keys (rk), 64..127 queries (rq)
+      // norms: half-row partial sums (threads 0..127 low halves, 128..255 high halves)
       {
-        const int r = t & 63;
-        const uint8_t* lo = rs + (t < 64 ? RS_KLO : RS_QLO);
-        const uint8_t* hi = rs + (t < 64 ? RS_KHI : RS_QHI);
+        const int nr = t & 127, part = t >> 7;
+        const uint8_t* tile = rs + (nr < 64 ? (part ? RS_KHI : RS_KLO) : (part ? RS_QHI : RS_QLO));
         float v[64];
         float sq = 0.f;
-        ptx::ld_row_bf16(lo, r, v);
+        ptx::ld_row_bf16(tile, nr & 63, v);
 #pragma unroll
         for (int e = 0; e < 64; ++e) sq = fmaf(v[e], v[e], sq);
-        ptx::ld_row_bf16(hi, r, v);
-#pragma unroll
-        for (int e = 0; e < 64; ++e) sq = fmaf(v[e], v[e], sq);
-        const bool valid = c0 + r < seq_end;
+        si[SI_NP + t] = sq;
+      }
+      named_bar_n(1, 256);
+      if (t < 128) {
+        const int nr = t & 63;
+        const float sq = si[SI_NP + t] + si[SI_NP + 128 + t];
+        const bool valid = c0t + nr < seq_end;
         float f = a.qk_l2norm ? 1.f / sqrtf(sq + kNormEps) : 1.f;
         if (t >= 64) f *= a.scale;
-        si[(t < 64 ? SI_RK : SI_RQ) + r] = valid ? f : 0.f;
+        si[(t < 64 ? SI_RK : SI_RQ) + nr] = valid ? f : 0.f;
       }
-      named_bar(1);
+      named_bar_n(1, 256);
       // GK[r][i] = rk_i exp(gcum_r - gcum_i) for i <= r (else 0); row scalars
 #pragma unroll 4
-      for (int e = t; e < 64 * 64; e += 128) {
-        const int r = e >> 6, i = e & 63;
-        const float val = (i <= r) ? si[SI_RK + i] * fast_exp(si[SI_GC + r] - si[SI_GC + i]) : 0.f;
-        gk[gk_index(r, i)] = val;
+      for (int e = t; e < 64 * 64; e += 256) {
+        const int gr = e >> 6, gi = e & 63;
+        const float val = (gi <= gr) ? si[SI_RK + gi] * fast_exp(si[SI_GC + gr] - si[SI_GC + gi]) : 0.f;
+        gk[gk_index(gr, gi)] = val;
       }
       if (t < 64) {
         const float gl = si[SI_GC + 63], gr = si[SI_GC + t];
@@ -318,50 +340,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       wait_mma();  // G ready (the named barrier inside also publishes GK)
       if (!ok) break;
-      // A rows + diagonal-block inverse (threads 0..63); P rows (threads 64..127)
-      float keep[64];  // key-row threads: R = T_D + N T_D, kept for T = R + N^2 R
-      float t16[16];   // key-row threads: strictly lower part of this row's T_D block
+      // A rows (key rows) with the diagonal-block inverse; P rows (query rows)
+      float keep[32];  // key rows: R = T_D + N T_D (this half), kept for T = R + N^2 R
+      float t16[16];   // diagonal-block threads: strictly lower part of this row's T_D block
       {
-        const int r = t & 63;
-        float av[64];
-        tmem_row64(tl + TM_G, av);
-        const float f = (t < 64) ? -si[SI_BETA + r] * si[SI_RK + r] : si[SI_RQ + r];
+        float av[32];
+        ptx::tmem_ld32(tl + TM_G + c0, av);
+        ptx::tmem_ld_wait();
+        const float f = krow ? -si[SI_BETA + r] * si[SI_RK + r] : si[SI_RQ + r];
         const float4* gkr = reinterpret_cast<const float4*>(gk + r * 64);
 #pragma unroll
-        for (int k4 = 0; k4 < 16; ++k4) {
-          const float4 x = gkr[k4 ^ (r & 7)];
+        for (int k4 = 0; k4 < 8; ++k4) {
+          const float4 x = gkr[(8 * hf + k4) ^ (r & 7)];
           av[4 * k4 + 0] *= f * x.x;
           av[4 * k4 + 1] *= f * x.y;
           av[4 * k4 + 2] *= f * x.z;
           av[4 * k4 + 3] *= f * x.w;
         }
-        if (t < 64) {
-          const int b = r >> 4, li = lane & 15;
+        if (krow) {
 #pragma unroll
-          for (int i = 0; i < 64; ++i) av[i] = (i == r) ? 0.f : av[i];  // strictly lower
+          for (int cc = 0; cc < 32; ++cc) av[cc] = (c0 + cc == r) ? 0.f : av[cc];  // strictly lower
+          if (diag_here) {
 #pragma unroll
-          for (int jj = 0; jj < 16; ++jj)
-            t16[jj] = (warp == 0) ? (lane < 16 ? av[jj] : av[16 + jj]) : (lane < 16 ? av[32 + jj] : av[48 + jj]);
+            for (int jj = 0; jj < 16; ++jj) t16[jj] = lane < 16 ? av[jj] : av[16 + jj];
 #pragma unroll
-          for (int m = 1; m < 15; ++m) {
-            const float coef = t16[m];
+            for (int m = 1; m < 15; ++m) {
+              const float coef = t16[m];
 #pragma unroll
-            for (int jj = 0; jj < m; ++jj) {
-              const float bj = __shfl_sync(0xffffffffu, t16[jj], (lane & 16) | m);
-              if (li > m) t16[jj] = fmaf(coef, bj, t16[jj]);
+              for (int jj = 0; jj < m; ++jj) {
+                const float bj = __shfl_sync(0xffffffffu, t16[jj], (lane & 16) | m);
+                if (li > m) t16[jj] = fmaf(coef, bj, t16[jj]);
+              }
             }
           }
+          td_half(t16, keep);
+          ptx::st_half_bf16(sm + OFF_X1, r, hf, keep);  // T_D
+          const int bcol = 16 * (r >> 4);
 #pragma unroll
-          for (int cc = 0; cc < 64; ++cc) {
-            const int cb = cc >> 4, cj = cc & 15;
-            keep[cc] = (cb == b) ? (cj < li ? t16[cj] : (cj == li ? 1.f : 0.f)) : 0.f;
-          }
-          ptx::st_row_bf16(sm + OFF_X1, r, keep);  // T_D
-#pragma unroll
-          for (int cc = 0; cc < 64; ++cc) av[cc] = (cc < 16 * b) ? av[cc] : 0.f;
-          ptx::st_row_bf16(sm + OFF_X0, r, av);  // A_off
+          for (int cc = 0; cc < 32; ++cc) av[cc] = (c0 + cc < bcol) ? av[cc] : 0.f;
+          ptx::st_half_bf16(sm + OFF_X0, r, hf, av);  // A_off
         } else {
-          ptx::st_row_bf16(ps + PS_P, r, av);  // P
+          ptx::st_half_bf16(ps + PS_P, r, hf, av);  // P
         }
       }
       publish();
@@ -373,10 +392,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       wait_mma();
       if (!ok) break;
-      if (t < 64) {
-        float x[64];
-        tmem_row64(tl + TM_G, x);
-        ptx::st_row_bf16(ps + PS_WLO, t, x);  // N (the GK table has been consumed)
+      if (krow) {
+        float x[32];
+        ptx::tmem_ld32(tl + TM_G + c0, x);
+        ptx::tmem_ld_wait();
+        ptx::st_half_bf16(ps + PS_WLO, r, hf, x);  // N (the GK table has been consumed)
       }
       publish();
       // [N^2 | N T_D] = N [N | T_D]
@@ -388,19 +408,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       wait_mma();
       if (!ok) break;
-      if (t < 64) {
-        const int r = t, b = r >> 4, li = lane & 15;
-        float x[64];
-        tmem_row64(tl + TM_N2, x);
-        ptx::st_row_bf16(sm + OFF_X0, r, x);  // N^2
-        tmem_row64(tl + TM_N2 + 64, x);
+      if (krow) {
+        float x[32];
+        ptx::tmem_ld32(tl + TM_N2 + c0, x);
+        ptx::tmem_ld_wait();
+        ptx::st_half_bf16(sm + OFF_X0, r, hf, x);  // N^2
+        ptx::tmem_ld32(tl + TM_N2 + 64 + c0, x);
+        ptx::tmem_ld_wait();
+        td_half(t16, keep);
 #pragma unroll
-        for (int cc = 0; cc < 64; ++cc) {
-          const int cb = cc >> 4, cj = cc & 15;
-          const float tdv = (cb == b) ? (cj < li ? t16[cj] : (cj == li ? 1.f : 0.f)) : 0.f;
-          keep[cc] = tdv + x[cc];  // R = T_D + N T_D
-        }
-        ptx::st_row_bf16(ps + PS_WHI, r, keep);
+        for (int cc = 0; cc < 32; ++cc) keep[cc] += x[cc];  // R = T_D + N T_D
+        ptx::st_half_bf16(ps + PS_WHI, r, hf, keep);
       }
       publish();
       // N^2 R
@@ -411,17 +429,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       wait_mma();
       if (!ok) break;
-      if (t < 64) {
-        float x[64];
-        tmem_row64(tl + TM_G, x);
+      if (krow) {
+        float x[32];
+        ptx::tmem_ld32(tl + TM_G + c0, x);
+        ptx::tmem_ld_wait();
 #pragma unroll
-        for (int cc = 0; cc < 64; ++cc) x[cc] += keep[cc];  // T = R + N^2 R
+        for (int cc = 0; cc < 32; ++cc) x[cc] += keep[cc];  // T = R + N^2 R
 #pragma unroll
-        for (int cc = 0; cc < 64; ++cc) keep[cc] = x[cc] * si[SI_BW + cc];
-        ptx::st_row_bf16(sm + OFF_X0, t, keep);  // T diag(beta exp(gcum) rk)
+        for (int cc = 0; cc < 32; ++cc) keep[cc] = x[cc] * si[SI_BW + c0 + cc];
+        ptx::st_half_bf16(sm + OFF_X0, r, hf, keep);  // T diag(beta exp(gcum) rk)
 #pragma unroll
-        for (int cc = 0; cc < 64; ++cc) keep[cc] = x[cc] * si[SI_BETA + cc];
-        ptx::st_row_bf16(ps + PS_TU, t, keep);  // T diag(beta), for U on the serial side
+        for (int cc = 0; cc < 32; ++cc) keep[cc] = x[cc] * si[SI_BETA + c0 + cc];
+        ptx::st_half_bf16(ps + PS_TU, r, hf, keep);  // T diag(beta), for U on the serial side
       }
       publish();
       // W = T diag(bw) K   (A = [T diag(bw); junk])
@@ -432,25 +451,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       wait_mma();
       if (!ok) break;
-      if (t < 64) {
+      if (krow) {
+        // W has 128 columns: this thread writes columns [64 hf, 64 hf + 64)
         float x[64];
-        tmem_row64(tl + TM_N2, x);
-        ptx::st_row_bf16(ps + PS_WLO, t, x);
-        tmem_row64(tl + TM_N2 + 64, x);
-        ptx::st_row_bf16(ps + PS_WHI, t, x);
+        ptx::tmem_ld32(tl + TM_N2 + 64 * hf, x);
+        ptx::tmem_ld32(tl + TM_N2 + 64 * hf + 32, x + 32);
+        ptx::tmem_ld_wait();
+        ptx::st_row_bf16(ps + (hf ? PS_WHI : PS_WLO), r, x);
       }
       publish();
       if (t == 0) ptx::mbar_arrive(bars + BAR_PRODF + psl);
       // tiles of chunk c + 2: their slot was used by chunk c - 1, which the
       // serial side has finished by now (it only lags this side by one chunk)
-      if (t == 96) prefetch(c + 2);
+      if (t == 224) prefetch(c + 2);
     }
     if (!ok && t == 0) atomicOr(&g_status, 1u);
   } else {
     // =====================================================================
-    // serial warpgroup
+    // serial warps (8-11)
     // =====================================================================
-    const int t = tid - 128;  // 0..127: row d of the state
+    const int t = tid - 256;  // 0..127: row d of the state
     float S[64];
     const size_t st_off = ((size_t)n * nv + h) * (size_t)DK * dv + (size_t)t * dv + slice * DVS;
     if (a.s0) {
@@ -466,13 +486,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     ptx::st_row_bf16(sm + OFF_S, t, S);
     ptx::fence_proxy_async_smem();
-    named_bar(2);
+    named_bar_n(2, 128);
 
     uint32_t ph_mma = 0;
     bool ok = true;
     auto wait_bar = [&](uint64_t* bar, uint32_t parity) {
       if (t == 0 && !ptx::mbar_wait_bounded(bar, parity, kWaitNs)) *abort_flag = 1;
-      named_bar(2);
+      named_bar_n(2, 128);
       ok = (*abort_flag == 0);
       ptx::tc_fence_after();
     };
@@ -483,13 +503,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto publish = [&]() {
       ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
-      named_bar(2);
+      named_bar_n(2, 128);
     };
 
-    float opart[64];  // lanes 64..127: diag(exp(gcum) rq) Q S
     for (int c = 0; c < nchunks && ok; ++c) {
       const int rsl = c % NR, psl = c % NP;
-      const int64_t c0 = seq_start + (int64_t)c * C;
+      const int64_t c0t = seq_start + (int64_t)c * C;
       const uint32_t ra = sb + OFF_RAW + rsl * kRaw;
       uint8_t* ps = sm + OFF_PROD + psl * kProd;
       const uint32_t pa = sb + OFF_PROD + psl * kProd;
@@ -507,22 +526,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       if (t < 64) {
         // V' = U - W S, and W' = diag(rk exp(g_last - gcum)) V'  (into the W tiles)
-        float u[64], ws[64];
-        tmem_row64(tl + TM_U, u);
-        tmem_row64(tl + TM_WS, ws);
-#pragma unroll
-        for (int cc = 0; cc < 64; ++cc) u[cc] -= ws[cc];
-        ptx::st_row_bf16(ps + PS_WLO, t, u);
         const float w = spp[SP_WK + t];
 #pragma unroll
-        for (int cc = 0; cc < 64; ++cc) u[cc] *= w;
-        ptx::st_row_bf16(ps + PS_WHI, t, u);
-      } else {
-        // Q S scaled by exp(gcum) rq, kept for the output
-        tmem_row64(tl + TM_KQS, opart);
-        const float f = spp[SP_SQ + t - 64];
+        for (int hh = 0; hh < 2; ++hh) {
+          float u[32], ws[32];
+          ptx::tmem_ld32(tl + TM_U + 32 * hh, u);
+          ptx::tmem_ld32(tl + TM_WS + 32 * hh, ws);
+          ptx::tmem_ld_wait();
 #pragma unroll
-        for (int cc = 0; cc < 64; ++cc) opart[cc] *= f;
+          for (int cc = 0; cc < 32; ++cc) u[cc] -= ws[cc];
+          ptx::st_half_bf16(ps + PS_WLO, t, hh, u);
+#pragma unroll
+          for (int cc = 0; cc < 32; ++cc) u[cc] *= w;
+          ptx::st_half_bf16(ps + PS_WHI, t, hh, u);
+        }
       }
       publish();
       // P V' (A = [junk; P]: rows land in lanes 64..127) and D4 = K^T W'
@@ -538,32 +555,41 @@ __global__ void __launch_bounds__(kThreads, 1)
       wait_mma();
       if (!ok) break;
       if (t >= 64) {
-        const int r = t - 64;
-        const int64_t tok = c0 + r;
-        float o[64];
-        tmem_row64(tl + TM_PV, o);
-        if (tok < seq_end) {
-          uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + ((size_t)tok * nv + h) * dv +
-                                                 slice * DVS);
+        // O = diag(exp(gcum) rq) Q S + P V'
+        const int orow = t - 64;
+        const int64_t tok = c0t + orow;
+        const float f = spp[SP_SQ + orow];
 #pragma unroll
-          for (int cc = 0; cc < 8; ++cc) {
-            const float* x = o + 8 * cc;
-            const float* y = opart + 8 * cc;
-            uint4 w;
-            w.x = ptx::pack_bf16x2(x[0] + y[0], x[1] + y[1]);
-            w.y = ptx::pack_bf16x2(x[2] + y[2], x[3] + y[3]);
-            w.z = ptx::pack_bf16x2(x[4] + y[4], x[5] + y[5]);
-            w.w = ptx::pack_bf16x2(x[6] + y[6], x[7] + y[7]);
-            orow[cc] = w;
+        for (int hh = 0; hh < 2; ++hh) {
+          float qs[32], pv[32];
+          ptx::tmem_ld32(tl + TM_KQS + 32 * hh, qs);
+          ptx::tmem_ld32(tl + TM_PV + 32 * hh, pv);
+          ptx::tmem_ld_wait();
+          if (tok < seq_end) {
+            uint4* op = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + ((size_t)tok * nv + h) * dv +
+                                                 slice * DVS + 32 * hh);
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+              uint4 w;
+              w.x = ptx::pack_bf16x2(fmaf(f, qs[8 * cc + 0], pv[8 * cc + 0]), fmaf(f, qs[8 * cc + 1], pv[8 * cc + 1]));
+              w.y = ptx::pack_bf16x2(fmaf(f, qs[8 * cc + 2], pv[8 * cc + 2]), fmaf(f, qs[8 * cc + 3], pv[8 * cc + 3]));
+              w.z = ptx::pack_bf16x2(fmaf(f, qs[8 * cc + 4], pv[8 * cc + 4]), fmaf(f, qs[8 * cc + 5], pv[8 * cc + 5]));
+              w.w = ptx::pack_bf16x2(fmaf(f, qs[8 * cc + 6], pv[8 * cc + 6]), fmaf(f, qs[8 * cc + 7], pv[8 * cc + 7]));
+              op[cc] = w;
+            }
           }
         }
       }
       {
         const float decay = spp[SP_GAMMA];
-        float x[64];
-        tmem_row64(tl + TM_D4, x);
 #pragma unroll
-        for (int cc = 0; cc < 64; ++cc) S[cc] = fmaf(decay, S[cc], x[cc]);
+        for (int hh = 0; hh < 2; ++hh) {
+          float x[32];
+          ptx::tmem_ld32(tl + TM_D4 + 32 * hh, x);
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int cc = 0; cc < 32; ++cc) S[32 * hh + cc] = fmaf(decay, S[32 * hh + cc], x[cc]);
+        }
         ptx::st_row_bf16(sm + OFF_S, t, S);
       }
       publish();

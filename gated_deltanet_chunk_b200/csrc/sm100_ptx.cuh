@@ -189,6 +189,19 @@ __device__ __forceinline__ void st_row_bf16(uint8_t* tile, int r, const float* v
   }
 }
 
+// Writes 32 fp32 values as the bf16 half (columns 32*half .. 32*half+31) of row r.
+__device__ __forceinline__ void st_half_bf16(uint8_t* tile, int r, int half, const float* v) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint4 w;
+    w.x = pack_bf16x2(v[8 * c + 0], v[8 * c + 1]);
+    w.y = pack_bf16x2(v[8 * c + 2], v[8 * c + 3]);
+    w.z = pack_bf16x2(v[8 * c + 4], v[8 * c + 5]);
+    w.w = pack_bf16x2(v[8 * c + 6], v[8 * c + 7]);
+    *reinterpret_cast<uint4*>(tile + sw128_off(r, 4 * half + c)) = w;
+  }
+}
+
 // Reads row r (64 bf16) of a swizzled tile into fp32.
 __device__ __forceinline__ void ld_row_bf16(const uint8_t* tile, int r, float* v) {
 #pragma unroll
