@@ -2,17 +2,20 @@
 //
 // bf16 q/k/v/out, Dk = Dv = 128, chunk C = 64.  One CTA owns one (sequence,
 // v-head, 64-column slice of Dv): the recurrence is separable in the Dv
-// columns.  Two warpgroups run a software pipeline over the sequence's chunks:
+// columns.  The two CTAs of a (sequence, v-head) form a cluster.  In each CTA:
 //
-//   intra warpgroup (warps 0-3): the state-independent part of chunk c -- gate
-//     cumsum, L2 norms, G = [K;Q] K^T, the A and P matrices, T = (I - A)^-1 and
-//     W -- runs ahead of the serial warpgroup.  Raw q/k/v tiles arrive by TMA
-//     in a ring of 3 input slots; the products (W, P, T diag(beta), per-row
-//     scalars) go to a ring of 2 product slots.
-//   serial warpgroup (warps 4-7): the state recurrence, two tensor-core round
-//     trips per chunk.  The fp32 state slice S [128 x 64] lives in registers
-//     (thread d holds row d) and, rounded to bf16, in shared memory as the B
-//     operand of the next chunk.
+//   intra warps (0-7): the state-independent part of a chunk -- gate cumsum,
+//     L2 norms, G = [K;Q] K^T, the A and P matrices, T = (I - A)^-1 and W.
+//     Chunk c is built only by cluster rank c % 2, which writes the products
+//     (W, P, T diag(beta), per-row scalars) into its own product slot and,
+//     through distributed shared memory, into the same slot of the other CTA,
+//     then releases them with a cluster-scope mbarrier arrive.  Each CTA thus
+//     builds every other chunk for both Dv slices.
+//   serial warps (8-11): the state recurrence for this CTA's Dv slice, two
+//     tensor-core round trips per chunk.  The fp32 state slice S [128 x 64]
+//     lives in registers (thread d holds row d) and, rounded to bf16, in shared
+//     memory as the B operand of the next chunk.  They also refill this CTA's
+//     3-deep TMA ring of raw q/k/v tiles.
 //
 // Algebra: the chunkwise form of the "手撕Qwen3-Next" walkthrough, section
 // 一(一)5(1), steps c-f, with the L2 norms folded into row scales
@@ -64,23 +67,26 @@ constexpr int kTile = 64 * 128;  // 64 rows x 128 bytes (64 bf16)
 // raw slot: [K_lo | Q_lo] [K_hi | Q_hi] V
 constexpr int RS_KLO = 0, RS_QLO = 1 * kTile, RS_KHI = 2 * kTile, RS_QHI = 3 * kTile, RS_V = 4 * kTile;
 constexpr int kRaw = 5 * kTile;
-// product slot: [W_lo | W_hi | P | T diag(beta)]; W_lo/W_hi hold the GK table
-// while the products are formed and V' / W' once the serial side has read W.
+// product slot: [W_lo | W_hi | P | T diag(beta)]; W_lo/W_hi hold V' / W' once
+// the serial side has read W.
 constexpr int PS_WLO = 0, PS_WHI = 1 * kTile, PS_P = 2 * kTile, PS_TU = 3 * kTile;
 constexpr int kProd = 4 * kTile;
 constexpr int OFF_RAW = 0;
 constexpr int OFF_PROD = NR * kRaw;
-constexpr int OFF_X0 = OFF_PROD + NP * kProd;  // intra scratch: A_off, N^2, T diag(bw)
-constexpr int OFF_X1 = OFF_X0 + kTile;         // intra scratch: T_D
+constexpr int OFF_X0 = OFF_PROD + NP * kProd;  // intra scratch: GK table (X0+X1), A_off, N, N^2, T diag(bw)
+constexpr int OFF_X1 = OFF_X0 + kTile;         // intra scratch: T_D, R
 constexpr int OFF_S = OFF_X1 + kTile;          // serial: S operand, 128 rows (d) x 64 cols
 constexpr int OFF_SCI = OFF_S + 2 * kTile;     // intra scalars
-constexpr int SI_RK = 0, SI_RQ = 64, SI_BETA = 128, SI_GC = 192, SI_BW = 256, SI_NP = 320, SI_N = 576;
+constexpr int SI_RK = 0, SI_RQ = 64, SI_BETA = 128, SI_GC = 192, SI_BW = 256, SI_NP = 320, SI_WK = 576,
+              SI_SQ = 640, SI_GAM = 704, SI_N = 708;
 constexpr int OFF_SCP = OFF_SCI + SI_N * 4;    // per-product-slot scalars for the serial side
 constexpr int SP_WK = 0, SP_SQ = 64, SP_GAMMA = 128, SP_N = 132;
 constexpr int OFF_BAR = OFF_SCP + NP * SP_N * 4;
-// barriers: raw_full[NR], raw_free[NR], prod_full[NP], prod_free[NP], mma_i, mma_s
-constexpr int BAR_RAWF = 0, BAR_RAWE = NR, BAR_PRODF = 2 * NR, BAR_PRODE = 2 * NR + NP;
-constexpr int BAR_MMAI = 2 * NR + 2 * NP, BAR_MMAS = BAR_MMAI + 1, NBAR = BAR_MMAS + 1;
+// barriers: raw_full[NR]; prod_full[NP] (the products of a chunk have landed in
+// this CTA); prod_free[NP] (this CTA's serial warps are done with the slot);
+// peer_free[NP] (the other CTA's serial warps are done with its copy); mma_i, mma_s
+constexpr int BAR_RAWF = 0, BAR_PRODF = NR, BAR_PRODE = NR + NP, BAR_PEERF = NR + 2 * NP;
+constexpr int BAR_MMAI = NR + 3 * NP, BAR_MMAS = BAR_MMAI + 1, NBAR = BAR_MMAS + 1;
 constexpr int SMEM_USED = OFF_BAR + NBAR * 8 + 16;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
 static_assert(OFF_BAR % 8 == 0, "mbarrier alignment");
@@ -158,14 +164,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   seq_bounds(a.cu, a.uniform_len, n, seq_start, seq_end);
   const int nchunks = (int)((seq_end - seq_start + C - 1) / C);
 
+  const uint32_t crank = ptx::cluster_ctarank();  // == slice
+  const uint32_t peer = crank ^ 1u;
   if (tid == 0) {
-    for (int i = 0; i < NR; ++i) {
-      ptx::mbar_init(bars + BAR_RAWF + i, 1);
-      ptx::mbar_init(bars + BAR_RAWE + i, 1);
-    }
+    for (int i = 0; i < NR; ++i) ptx::mbar_init(bars + BAR_RAWF + i, 1);
     for (int i = 0; i < NP; ++i) {
       ptx::mbar_init(bars + BAR_PRODF + i, 1);
       ptx::mbar_init(bars + BAR_PRODE + i, 1);
+      ptx::mbar_init(bars + BAR_PEERF + i, 1);
     }
     ptx::mbar_init(bars + BAR_MMAI, 1);
     ptx::mbar_init(bars + BAR_MMAS, 1);
@@ -181,6 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   ptx::tc_fence_before();
   __syncthreads();
+  ptx::cluster_sync_all();  // both CTAs' barriers are initialised before any remote arrive
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);  // this warp's TMEM lane quarter
@@ -200,18 +207,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the 16x16 diagonal block of key row r lies in this thread's half
     const bool diag_here = krow && ((r >> 5) == hf);
     const int li = lane & 15;
-    auto issue_tma = [&](int chunk) {
-      const int s = chunk % NR;
-      const int t0 = (int)(seq_start + (int64_t)chunk * C);
-      uint8_t* rs = sm + OFF_RAW + s * kRaw;
-      uint64_t* bar = bars + BAR_RAWF + s;
-      ptx::mbar_arrive_expect_tx(bar, 5 * kTile);
-      ptx::tma_load_3d(rs + RS_KLO, &tm_k, bar, 0, j, t0);
-      ptx::tma_load_3d(rs + RS_KHI, &tm_k, bar, 64, j, t0);
-      ptx::tma_load_3d(rs + RS_QLO, &tm_q, bar, 0, j, t0);
-      ptx::tma_load_3d(rs + RS_QHI, &tm_q, bar, 64, j, t0);
-      ptx::tma_load_3d(rs + RS_V, &tm_v, bar, slice * DVS, h, t0);
-    };
     uint32_t ph_mma = 0;
     bool ok = true;
     // One thread polls the mbarrier; the others park at the named barrier.
@@ -230,13 +225,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::tc_fence_before();
       named_bar_n(1, 256);
     };
-    // The raw slot of chunk c' becomes free when the serial side has finished chunk c' - NR.
-    auto prefetch = [&](int cn) {
-      if (cn >= nchunks) return;
-      if (cn >= NR && !ptx::mbar_wait_bounded(bars + BAR_RAWE + cn % NR, (uint32_t)((cn / NR - 1) & 1), kWaitNs))
-        *abort_flag = 1;
-      issue_tma(cn);
-    };
     // this thread's 32 columns of T_D (block-diagonal inverse) for key row r
     auto td_half = [&](const float* t16, float* out32) {
 #pragma unroll
@@ -247,17 +235,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     };
 
-    if (t == 224) {  // a query-row warp issues the tensor loads
-      prefetch(0);
-      prefetch(1);
-    }
     float g_next = 0.f, b_next = 0.f;
-    if (t < 64 && seq_start + t < seq_end) {
-      g_next = a.g[(size_t)(seq_start + t) * nv + h];
-      b_next = a.beta[(size_t)(seq_start + t) * nv + h];
+    {
+      const int64_t t0g = seq_start + (int64_t)crank * C + t;
+      if (t < 64 && t0g < seq_end) {
+        g_next = a.g[(size_t)t0g * nv + h];
+        b_next = a.beta[(size_t)t0g * nv + h];
+      }
     }
 
-    for (int c = 0; c < nchunks && ok; ++c) {
+    // this CTA builds the chunks c with c % 2 == cluster rank
+    for (int c = (int)crank; c < nchunks && ok; c += 2) {
       const int rsl = c % NR, psl = c % NP;
       const int64_t c0t = seq_start + (int64_t)c * C;
       uint8_t* rs = sm + OFF_RAW + rsl * kRaw;
@@ -265,7 +253,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint8_t* ps = sm + OFF_PROD + psl * kProd;
       const uint32_t pa = sb + OFF_PROD + psl * kProd;
       float* spp = sp + psl * SP_N;
-      float* gk = reinterpret_cast<float*>(ps + PS_WLO);  // 16 KB: the W_lo / W_hi tiles
+      float* gk = reinterpret_cast<float*>(sm + OFF_X0);  // 16 KB: the X0 / X1 scratch tiles
+      const uint32_t rpa = ptx::mapa(pa, peer);                     // the other CTA's copy of the slot
+      const uint32_t rspp = ptx::mapa(ptx::smem_u32(spp), peer);
 
       // gates: beta and the warp-local cumsum of g; prefetch the next chunk's gates
       if (t < 64) {
@@ -277,7 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane >= o) gv += y;
         }
         si[SI_GC + t] = gv;
-        const int64_t tn = c0t + C + t;
+        const int64_t tn = c0t + 2 * C + t;  // this CTA's next chunk
         g_next = 0.f;
         b_next = 0.f;
         if (tn < seq_end) {
@@ -285,10 +275,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           b_next = a.beta[(size_t)tn * nv + h];
         }
       }
-      // the product slot must have been released by the serial side (chunk c - NP)
-      if (t == 0 && c >= NP &&
-          !ptx::mbar_wait_bounded(bars + BAR_PRODE + psl, (uint32_t)((c / NP - 1) & 1), kWaitNs))
-        *abort_flag = 1;
       wait_bar(bars + BAR_RAWF + rsl, (uint32_t)((c / NR) & 1));
       if (!ok) break;
       // G = [K; Q] K^T
@@ -334,14 +320,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float eg = fast_exp(gr);
         const float rk = si[SI_RK + t];
         si[SI_BW + t] = si[SI_BETA + t] * eg * rk;
-        spp[SP_WK + t] = rk * fast_exp(gl - gr);
-        spp[SP_SQ + t] = eg * si[SI_RQ + t];
-        if (t == 0) spp[SP_GAMMA] = fast_exp(gl);
+        si[SI_WK + t] = rk * fast_exp(gl - gr);
+        si[SI_SQ + t] = eg * si[SI_RQ + t];
+        if (t == 0) si[SI_GAM] = fast_exp(gl);
       }
       wait_mma();  // G ready (the named barrier inside also publishes GK)
       if (!ok) break;
       // A rows (key rows) with the diagonal-block inverse; P rows (query rows)
-      float keep[32];  // key rows: R = T_D + N T_D (this half), kept for T = R + N^2 R
+      float keep[32];  // key rows: R = T_D + N T_D (this half); query rows: this half of P
       float t16[16];   // diagonal-block threads: strictly lower part of this row's T_D block
       {
         float av[32];
@@ -357,6 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           av[4 * k4 + 2] *= f * x.z;
           av[4 * k4 + 3] *= f * x.w;
         }
+        named_bar_n(1, 256);  // every GK row has been read: X0 / X1 are free
         if (krow) {
 #pragma unroll
           for (int cc = 0; cc < 32; ++cc) av[cc] = (c0 + cc == r) ? 0.f : av[cc];  // strictly lower
@@ -380,7 +367,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int cc = 0; cc < 32; ++cc) av[cc] = (c0 + cc < bcol) ? av[cc] : 0.f;
           ptx::st_half_bf16(sm + OFF_X0, r, hf, av);  // A_off
         } else {
-          ptx::st_half_bf16(ps + PS_P, r, hf, av);  // P
+#pragma unroll
+          for (int cc = 0; cc < 32; ++cc) keep[cc] = av[cc];  // P, stored once the slot is free
         }
       }
       publish();
@@ -396,14 +384,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         float x[32];
         ptx::tmem_ld32(tl + TM_G + c0, x);
         ptx::tmem_ld_wait();
-        ptx::st_half_bf16(ps + PS_WLO, r, hf, x);  // N (the GK table has been consumed)
+        ptx::st_half_bf16(sm + OFF_X0, r, hf, x);  // N (A_off has been consumed)
       }
       publish();
       // [N^2 | N T_D] = N [N | T_D]
       if (t == 0) {
         ptx::tc_fence_after();
-        mma_k64(tmem + TM_N2, pa + PS_WLO, pa + PS_WLO, (uint32_t)(OFF_X1 - (OFF_PROD + psl * kProd + PS_WLO)),
-                ID_KMN128, 0);
+        mma_k64(tmem + TM_N2, sb + OFF_X0, sb + OFF_X0, OFF_X1 - OFF_X0, ID_KMN128, 0);
         ptx::mma_commit(bars + BAR_MMAI);
       }
       wait_mma();
@@ -418,17 +405,42 @@ __global__ void __launch_bounds__(kThreads, 1)
         td_half(t16, keep);
 #pragma unroll
         for (int cc = 0; cc < 32; ++cc) keep[cc] += x[cc];  // R = T_D + N T_D
-        ptx::st_half_bf16(ps + PS_WHI, r, hf, keep);
+        ptx::st_half_bf16(sm + OFF_X1, r, hf, keep);  // R (T_D has been consumed)
       }
       publish();
       // N^2 R
       if (t == 0) {
         ptx::tc_fence_after();
-        mma_k64(tmem + TM_G, sb + OFF_X0, pa + PS_WHI, 8192, ID_KMN64, 0);
+        mma_k64(tmem + TM_G, sb + OFF_X0, sb + OFF_X1, 8192, ID_KMN64, 0);
         ptx::mma_commit(bars + BAR_MMAI);
       }
-      wait_mma();
+      // the product slot (both copies) must have been released by both CTAs'
+      // serial warps (chunk c - 2) before the products are stored
+      if (t == 0) {
+        if (!ptx::mbar_wait_bounded(bars + BAR_MMAI, ph_mma, kWaitNs)) *abort_flag = 1;
+        if (c >= NP) {
+          const uint32_t par = (uint32_t)((c / NP - 1) & 1);
+          if (!ptx::mbar_wait_bounded(bars + BAR_PRODE + psl, par, kWaitNs)) *abort_flag = 1;
+          if (!ptx::mbar_wait_cluster_bounded(bars + BAR_PEERF + psl, par, kWaitNs)) *abort_flag = 1;
+        }
+      }
+      ph_mma ^= 1u;
+      named_bar_n(1, 256);
+      ok = (*abort_flag == 0);
+      ptx::tc_fence_after();
       if (!ok) break;
+      if (t < 64) {
+        const float wk = si[SI_WK + t], sq = si[SI_SQ + t];
+        spp[SP_WK + t] = wk;
+        spp[SP_SQ + t] = sq;
+        ptx::st_cluster_f32(rspp + 4 * (SP_WK + t), wk);
+        ptx::st_cluster_f32(rspp + 4 * (SP_SQ + t), sq);
+        if (t == 0) {
+          spp[SP_GAMMA] = si[SI_GAM];
+          ptx::st_cluster_f32(rspp + 4 * SP_GAMMA, si[SI_GAM]);
+        }
+      }
+      if (!krow) ptx::st_half_bf16_dual(ps + PS_P, rpa + PS_P, r, hf, keep);  // P
       if (krow) {
         float x[32];
         ptx::tmem_ld32(tl + TM_G + c0, x);
@@ -440,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::st_half_bf16(sm + OFF_X0, r, hf, keep);  // T diag(beta exp(gcum) rk)
 #pragma unroll
         for (int cc = 0; cc < 32; ++cc) keep[cc] = x[cc] * si[SI_BETA + c0 + cc];
-        ptx::st_half_bf16(ps + PS_TU, r, hf, keep);  // T diag(beta), for U on the serial side
+        ptx::st_half_bf16_dual(ps + PS_TU, rpa + PS_TU, r, hf, keep);  // T diag(beta), for U
       }
       publish();
       // W = T diag(bw) K   (A = [T diag(bw); junk])
@@ -457,13 +469,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::tmem_ld32(tl + TM_N2 + 64 * hf, x);
         ptx::tmem_ld32(tl + TM_N2 + 64 * hf + 32, x + 32);
         ptx::tmem_ld_wait();
-        ptx::st_row_bf16(ps + (hf ? PS_WHI : PS_WLO), r, x);
+        ptx::st_row_bf16_dual(ps + (hf ? PS_WHI : PS_WLO), rpa + (hf ? PS_WHI : PS_WLO), r, x);
       }
+      ptx::fence_acq_rel_cluster();  // remote product stores before the release below
       publish();
-      if (t == 0) ptx::mbar_arrive(bars + BAR_PRODF + psl);
-      // tiles of chunk c + 2: their slot was used by chunk c - 1, which the
-      // serial side has finished by now (it only lags this side by one chunk)
-      if (t == 224) prefetch(c + 2);
+      if (t == 0) {
+        ptx::mbar_arrive(bars + BAR_PRODF + psl);
+        ptx::mbar_arrive_remote(ptx::mapa(ptx::smem_u32(bars + BAR_PRODF + psl), peer));
+      }
     }
     if (!ok && t == 0) atomicOr(&g_status, 1u);
   } else {
@@ -496,6 +509,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = (*abort_flag == 0);
       ptx::tc_fence_after();
     };
+    // this CTA's raw q/k/v tiles of chunk `chunk` (slot chunk % NR)
+    auto issue_tma = [&](int chunk) {
+      const int s = chunk % NR;
+      const int t0 = (int)(seq_start + (int64_t)chunk * C);
+      uint8_t* rs = sm + OFF_RAW + s * kRaw;
+      uint64_t* bar = bars + BAR_RAWF + s;
+      ptx::mbar_arrive_expect_tx(bar, 5 * kTile);
+      ptx::tma_load_3d(rs + RS_KLO, &tm_k, bar, 0, j, t0);
+      ptx::tma_load_3d(rs + RS_KHI, &tm_k, bar, 64, j, t0);
+      ptx::tma_load_3d(rs + RS_QLO, &tm_q, bar, 0, j, t0);
+      ptx::tma_load_3d(rs + RS_QHI, &tm_q, bar, 64, j, t0);
+      ptx::tma_load_3d(rs + RS_V, &tm_v, bar, slice * DVS, h, t0);
+    };
+    int issued = 0;    // chunks whose tiles have been requested
+    int consumed = 0;  // chunks whose tiles this warpgroup has waited for
+    if (t == 64)
+      for (; issued < NR && issued < nchunks; ++issued) issue_tma(issued);
     auto wait_mma = [&]() {
       wait_bar(bars + BAR_MMAS, ph_mma);
       ph_mma ^= 1u;
@@ -513,10 +543,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint8_t* ps = sm + OFF_PROD + psl * kProd;
       const uint32_t pa = sb + OFF_PROD + psl * kProd;
       const float* spp = sp + psl * SP_N;
-      wait_bar(bars + BAR_PRODF + psl, (uint32_t)((c / NP) & 1));
+      // this CTA's tiles, then the products (built here or by the other CTA)
+      if (t == 0) {
+        if (!ptx::mbar_wait_bounded(bars + BAR_RAWF + rsl, (uint32_t)((c / NR) & 1), kWaitNs)) *abort_flag = 1;
+        if (!ptx::mbar_wait_cluster_bounded(bars + BAR_PRODF + psl, (uint32_t)((c / NP) & 1), kWaitNs))
+          *abort_flag = 1;
+      }
+      named_bar_n(2, 128);
+      ok = (*abort_flag == 0);
+      ptx::tc_fence_after();
       if (!ok) break;
+      consumed = c + 1;
       // [K S; Q S],  W S (A = [W; junk]),  U = T diag(beta) V (A = [Tb; junk])
       if (t == 0) {
+        ptx::fence_proxy_async_smem();  // products stored by threads (possibly of the other CTA)
         mma_k128(tmem + TM_KQS, ra + RS_KLO, ra + RS_KHI, sb + OFF_S, 8192, ID_KMN64);
         mma_k128(tmem + TM_WS, pa + PS_WLO, pa + PS_WHI, sb + OFF_S, 8192, ID_KMN64);
         mma_k64(tmem + TM_U, pa + PS_TU, ra + RS_V, 8192, ID_KMN64, 0);
@@ -593,10 +633,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::st_row_bf16(sm + OFF_S, t, S);
       }
       publish();
-      if (t == 0) {
-        ptx::mbar_arrive(bars + BAR_PRODE + psl);
-        ptx::mbar_arrive(bars + BAR_RAWE + rsl);
+      if (t == 64) {  // off the polling thread's path
+        // release the product slot to the CTA that builds chunk c + 2
+        if ((c & 1) == (int)crank)
+          ptx::mbar_arrive(bars + BAR_PRODE + psl);
+        else
+          ptx::mbar_arrive_remote(ptx::mapa(ptx::smem_u32(bars + BAR_PEERF + psl), peer));
+        if (c + NR < nchunks) {  // every read of this raw slot has completed
+          issue_tma(c + NR);
+          issued = c + NR + 1;
+        }
       }
+    }
+    if (!ok && t == 64) {
+      // abort: let the tile loads still in flight land before this CTA exits (bounded)
+      for (int cn = consumed; cn < issued; ++cn)
+        ptx::mbar_wait_bounded(bars + BAR_RAWF + cn % NR, (uint32_t)((cn / NR) & 1), kWaitNs);
     }
     if (ok && a.s_final) {
       float4* dst = reinterpret_cast<float4*>(a.s_final + st_off);
@@ -608,6 +660,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   ptx::tc_fence_before();
   __syncthreads();
+  ptx::cluster_sync_all();  // the other CTA no longer touches this CTA's shared memory
   if (warp == 0) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, TM_COLS);
@@ -655,8 +708,20 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int64_t total_tokens, cudaStream
   cudaError_t e = cudaFuncSetAttribute(tc::chunk_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        tc::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  dim3 grid(a.dv / tc::DVS, a.nv, a.num_seqs);
-  tc::chunk_fwd_tc_kernel<<<grid, tc::kThreads, tc::SMEM_BYTES, stream>>>(mq, mk, mv, a);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.dv / tc::DVS, a.nv, a.num_seqs);  // x: the two Dv slices = one cluster
+  cfg.blockDim = dim3(tc::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = tc::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, tc::chunk_fwd_tc_kernel, mq, mk, mv, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -76,6 +76,58 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
+// ------------------------------------------------------------------ clusters / DSMEM
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// shared::cluster address of the same shared-memory offset in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t mapa(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+// arrive on an mbarrier of another CTA of the cluster; orders this thread's prior
+// (and, cumulatively, observed) writes before it at cluster scope
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// bounded wait with cluster-scope acquire (for phases completed by another CTA)
+__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+__device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
                                             int c2) {
@@ -199,6 +251,37 @@ __device__ __forceinline__ void st_half_bf16(uint8_t* tile, int r, int half, con
     w.z = pack_bf16x2(v[8 * c + 4], v[8 * c + 5]);
     w.w = pack_bf16x2(v[8 * c + 6], v[8 * c + 7]);
     *reinterpret_cast<uint4*>(tile + sw128_off(r, 4 * half + c)) = w;
+  }
+}
+
+// Packs 8 fp32 values (v[0..7]) into one 16-byte bf16 chunk.
+__device__ __forceinline__ uint4 pack8_bf16(const float* v) {
+  uint4 w;
+  w.x = pack_bf16x2(v[0], v[1]);
+  w.y = pack_bf16x2(v[2], v[3]);
+  w.z = pack_bf16x2(v[4], v[5]);
+  w.w = pack_bf16x2(v[6], v[7]);
+  return w;
+}
+
+// Like st_half_bf16 / st_row_bf16, also storing the same bytes to `remote`,
+// the shared::cluster address of the same tile in another CTA of the cluster.
+__device__ __forceinline__ void st_half_bf16_dual(uint8_t* tile, uint32_t remote, int r, int half, const float* v) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const uint4 w = pack8_bf16(v + 8 * c);
+    const uint32_t off = sw128_off(r, 4 * half + c);
+    *reinterpret_cast<uint4*>(tile + off) = w;
+    st_cluster_v4(remote + off, w);
+  }
+}
+__device__ __forceinline__ void st_row_bf16_dual(uint8_t* tile, uint32_t remote, int r, const float* v) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const uint4 w = pack8_bf16(v + 8 * c);
+    const uint32_t off = sw128_off(r, c);
+    *reinterpret_cast<uint4*>(tile + off) = w;
+    st_cluster_v4(remote + off, w);
   }
 }
 
