@@ -8,14 +8,16 @@
 //     L2 norms, G = [K;Q] K^T, the A and P matrices, T = (I - A)^-1 and W.
 //     Chunk c is built only by cluster rank c % 2, which writes the products
 //     (W, P, T diag(beta), per-row scalars) into its own product slot and,
-//     through distributed shared memory, into the same slot of the other CTA,
-//     then releases them with a cluster-scope mbarrier arrive.  Each CTA thus
-//     builds every other chunk for both Dv slices.
-//   serial warps (8-11): the state recurrence for this CTA's Dv slice, two
-//     tensor-core round trips per chunk.  The fp32 state slice S [128 x 64]
-//     lives in registers (thread d holds row d) and, rounded to bf16, in shared
-//     memory as the B operand of the next chunk.  They also refill this CTA's
-//     3-deep TMA ring of raw q/k/v tiles.
+//     with st.async into distributed shared memory, into the same slot of the
+//     other CTA, whose mbarrier completes when all those bytes have landed.
+//     Each CTA thus builds every other chunk for both Dv slices.
+//   serial warps (8-11): the state recurrence for this CTA's Dv slice.  The
+//     fp32 state slice S [128 x 64] lives in registers (thread d holds row d)
+//     and, rounded to bf16, in shared memory as the B operand of the next
+//     chunk.  The critical path per chunk is two tensor-core round trips
+//     (U - W S, then D4) and two short epilogues; the output rows (P V' + Q S)
+//     are finished by warps 10-11 while warps 8-9 start the next chunk.  The
+//     serial warps also refill this CTA's 3-deep TMA ring of raw q/k/v tiles.
 //
 // Algebra: the chunkwise form of the "手撕Qwen3-Next" walkthrough, section
 // 一(一)5(1), steps c-f, with the L2 norms folded into row scales
@@ -29,11 +31,12 @@
 //        (T_D: inverse of A's 16x16 diagonal blocks by forward substitution
 //        in registers; A_off: the strictly block-lower part of A; N^4 = 0.
 //        The 16-row block scheme is the PyPTO README's inverse_pto submodule.)
-//   W  = T diag(beta exp(gcum) rk) K                                    tcgen05
-//   serial:  [KS; QS] = [K; Q] S,  WS = W S,  U = T diag(beta) V        one round
-//            V' = U - W S                                               CUDA cores
-//            PV = P V',  D4 = K^T diag(rk exp(g_last - gcum)) V'        one round
-//            O = diag(exp(gcum) rq) QS + PV;  S <- exp(g_last) S + D4
+//   W  = T diag(beta exp(gcum) rk) K  (stored negated)                  tcgen05
+//   serial:  V' = T diag(beta) V + (-W) S   (one accumulator)           one round
+//            [KS; QS] = [K; Q] S                                  same round, own use
+//            D4 = K^T diag(rk exp(g_last - gcum)) V'                    one round
+//            PV = P V'                                            after D4, own use
+//            S <- exp(g_last) S + D4;  O = diag(exp(gcum) rq) QS + PV
 // Every accumulation is fp32 in TMEM; MMA operands are bf16.
 //
 // Operand placement: an M=128 A operand is two stacked 64-row tiles; where only
@@ -81,12 +84,15 @@ constexpr int SI_RK = 0, SI_RQ = 64, SI_BETA = 128, SI_GC = 192, SI_BW = 256, SI
               SI_SQ = 640, SI_GAM = 704, SI_N = 708;
 constexpr int OFF_SCP = OFF_SCI + SI_N * 4;    // per-product-slot scalars for the serial side
 constexpr int SP_WK = 0, SP_SQ = 64, SP_GAMMA = 128, SP_N = 132;
+// bytes one CTA sends to the other per chunk it builds: W, P, T diag(beta), wk, sq, gamma
+constexpr uint32_t kPushBytes = 4 * 8192 + (2 * 64 + 1) * 4;
 constexpr int OFF_BAR = OFF_SCP + NP * SP_N * 4;
 // barriers: raw_full[NR]; prod_full[NP] (the products of a chunk have landed in
 // this CTA); prod_free[NP] (this CTA's serial warps are done with the slot);
 // peer_free[NP] (the other CTA's serial warps are done with its copy); mma_i, mma_s
 constexpr int BAR_RAWF = 0, BAR_PRODF = NR, BAR_PRODE = NR + NP, BAR_PEERF = NR + 2 * NP;
-constexpr int BAR_MMAI = NR + 3 * NP, BAR_MMAS = BAR_MMAI + 1, NBAR = BAR_MMAS + 1;
+constexpr int BAR_MMAI = NR + 3 * NP, BAR_MMAS = BAR_MMAI + 1, BAR_MMAD4 = BAR_MMAS + 1, BAR_MMAO = BAR_MMAD4 + 1;
+constexpr int BAR_OUTD = BAR_MMAO + 1, NBAR = BAR_OUTD + 1;
 constexpr int SMEM_USED = OFF_BAR + NBAR * 8 + 16;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
 static_assert(OFF_BAR % 8 == 0, "mbarrier alignment");
@@ -95,9 +101,8 @@ static_assert(SMEM_BYTES <= 232448, "shared memory");
 // ---- TMEM columns (128 lanes x 512 fp32 columns)
 constexpr uint32_t TM_G = 0;     // intra: G; then N; then N^2 R
 constexpr uint32_t TM_N2 = 64;   // intra: [N^2 | N T_D] (128 cols); then W (128 cols)
-constexpr uint32_t TM_KQS = 192; // serial: [K S ; Q S]
-constexpr uint32_t TM_WS = 256;  // serial: W S (rows 0..63)
-constexpr uint32_t TM_U = 320;   // serial: U (rows 0..63)
+constexpr uint32_t TM_QS = 192;  // serial: [K S ; Q S], two column blocks used alternately (128 cols)
+constexpr uint32_t TM_U = 320;   // serial: U - W S (rows 0..63)
 constexpr uint32_t TM_PV = 384;  // serial: P V' (rows 64..127)
 constexpr uint32_t TM_D4 = 448;  // serial: state update
 constexpr uint32_t TM_COLS = 512;
@@ -121,10 +126,11 @@ __device__ __forceinline__ void mma_k64(uint32_t d, uint32_t a, uint32_t b, uint
 
 // K = 128 product: A K-major split in two 64-column tiles at a_lo / a_hi, B MN-major at b.
 __device__ __forceinline__ void mma_k128(uint32_t d, uint32_t a_lo, uint32_t a_hi, uint32_t b, uint32_t b_lbo,
-                                         uint32_t idesc) {
+                                         uint32_t idesc, uint32_t acc) {
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk)
-    ptx::mma_bf16(d, kdesc((kk < 4 ? a_lo : a_hi) + 32 * (kk & 3)), mndesc(b + 2048 * kk, b_lbo), idesc, kk > 0);
+    ptx::mma_bf16(d, kdesc((kk < 4 ? a_lo : a_hi) + 32 * (kk & 3)), mndesc(b + 2048 * kk, b_lbo), idesc,
+                  acc | (kk > 0));
 }
 
 __device__ __forceinline__ void tmem_row64(uint32_t taddr, float* v) {
@@ -135,6 +141,22 @@ __device__ __forceinline__ void tmem_row64(uint32_t taddr, float* v) {
 
 __device__ __forceinline__ void named_bar_n(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Named barrier that also ORs `flag` over the participating threads: every
+// participant gets the same answer, so a loop exit decided on it is uniform
+// even while another role may be setting the abort flag.
+__device__ __forceinline__ bool named_bar_any(int id, int nthreads, bool flag) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)flag), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
 }
 
 // GK table: fp32 [64][64], rows of 256 bytes with the 16-byte chunk k of row r
@@ -175,6 +197,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     ptx::mbar_init(bars + BAR_MMAI, 1);
     ptx::mbar_init(bars + BAR_MMAS, 1);
+    ptx::mbar_init(bars + BAR_MMAD4, 1);
+    ptx::mbar_init(bars + BAR_MMAO, 1);
+    ptx::mbar_init(bars + BAR_OUTD, 2);
     *abort_flag = 0;
     ptx::fence_mbar_init();
     ptx::prefetch_tensormap(&tm_q);
@@ -212,8 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // One thread polls the mbarrier; the others park at the named barrier.
     auto wait_bar = [&](uint64_t* bar, uint32_t parity) {
       if (t == 0 && !ptx::mbar_wait_bounded(bar, parity, kWaitNs)) *abort_flag = 1;
-      named_bar_n(1, 256);
-      ok = (*abort_flag == 0);
+      ok = !named_bar_any(1, 256, *abort_flag != 0);
       ptx::tc_fence_after();
     };
     auto wait_mma = [&]() {
@@ -256,6 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float* gk = reinterpret_cast<float*>(sm + OFF_X0);  // 16 KB: the X0 / X1 scratch tiles
       const uint32_t rpa = ptx::mapa(pa, peer);                     // the other CTA's copy of the slot
       const uint32_t rspp = ptx::mapa(ptx::smem_u32(spp), peer);
+      const uint32_t rbar = ptx::mapa(ptx::smem_u32(bars + BAR_PRODF + psl), peer);  // the other CTA's prod_full
 
       // gates: beta and the warp-local cumsum of g; prefetch the next chunk's gates
       if (t < 64) {
@@ -423,24 +448,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ptx::mbar_wait_bounded(bars + BAR_PRODE + psl, par, kWaitNs)) *abort_flag = 1;
           if (!ptx::mbar_wait_cluster_bounded(bars + BAR_PEERF + psl, par, kWaitNs)) *abort_flag = 1;
         }
+        if (*abort_flag == 0) ptx::mbar_arrive_expect_tx_remote(rbar, kPushBytes);  // arm the other CTA's copy
       }
       ph_mma ^= 1u;
-      named_bar_n(1, 256);
-      ok = (*abort_flag == 0);
+      ok = !named_bar_any(1, 256, *abort_flag != 0);
       ptx::tc_fence_after();
       if (!ok) break;
       if (t < 64) {
         const float wk = si[SI_WK + t], sq = si[SI_SQ + t];
         spp[SP_WK + t] = wk;
         spp[SP_SQ + t] = sq;
-        ptx::st_cluster_f32(rspp + 4 * (SP_WK + t), wk);
-        ptx::st_cluster_f32(rspp + 4 * (SP_SQ + t), sq);
+        ptx::st_async_b32(rspp + 4 * (SP_WK + t), __float_as_uint(wk), rbar);
+        ptx::st_async_b32(rspp + 4 * (SP_SQ + t), __float_as_uint(sq), rbar);
         if (t == 0) {
           spp[SP_GAMMA] = si[SI_GAM];
-          ptx::st_cluster_f32(rspp + 4 * SP_GAMMA, si[SI_GAM]);
+          ptx::st_async_b32(rspp + 4 * SP_GAMMA, __float_as_uint(si[SI_GAM]), rbar);
         }
       }
-      if (!krow) ptx::st_half_bf16_dual(ps + PS_P, rpa + PS_P, r, hf, keep);  // P
+      if (!krow) ptx::st_half_bf16_dual(ps + PS_P, rpa + PS_P, rbar, r, hf, keep);  // P
       if (krow) {
         float x[32];
         ptx::tmem_ld32(tl + TM_G + c0, x);
@@ -452,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::st_half_bf16(sm + OFF_X0, r, hf, keep);  // T diag(beta exp(gcum) rk)
 #pragma unroll
         for (int cc = 0; cc < 32; ++cc) keep[cc] = x[cc] * si[SI_BETA + c0 + cc];
-        ptx::st_half_bf16_dual(ps + PS_TU, rpa + PS_TU, r, hf, keep);  // T diag(beta), for U
+        ptx::st_half_bf16_dual(ps + PS_TU, rpa + PS_TU, rbar, r, hf, keep);  // T diag(beta), for U
       }
       publish();
       // W = T diag(bw) K   (A = [T diag(bw); junk])
@@ -469,14 +494,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::tmem_ld32(tl + TM_N2 + 64 * hf, x);
         ptx::tmem_ld32(tl + TM_N2 + 64 * hf + 32, x + 32);
         ptx::tmem_ld_wait();
-        ptx::st_row_bf16_dual(ps + (hf ? PS_WHI : PS_WLO), rpa + (hf ? PS_WHI : PS_WLO), r, x);
+#pragma unroll
+        for (int cc = 0; cc < 64; ++cc) x[cc] = -x[cc];  // the serial side accumulates U + (-W) S
+        ptx::st_row_bf16_dual(ps + (hf ? PS_WHI : PS_WLO), rpa + (hf ? PS_WHI : PS_WLO), rbar, r, x);
       }
-      ptx::fence_acq_rel_cluster();  // remote product stores before the release below
       publish();
-      if (t == 0) {
-        ptx::mbar_arrive(bars + BAR_PRODF + psl);
-        ptx::mbar_arrive_remote(ptx::mapa(ptx::smem_u32(bars + BAR_PRODF + psl), peer));
-      }
+      if (t == 0) ptx::mbar_arrive(bars + BAR_PRODF + psl);  // the other CTA's copy completes by transactions
     }
     if (!ok && t == 0) atomicOr(&g_status, 1u);
   } else {
@@ -501,14 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::fence_proxy_async_smem();
     named_bar_n(2, 128);
 
-    uint32_t ph_mma = 0;
     bool ok = true;
-    auto wait_bar = [&](uint64_t* bar, uint32_t parity) {
-      if (t == 0 && !ptx::mbar_wait_bounded(bar, parity, kWaitNs)) *abort_flag = 1;
-      named_bar_n(2, 128);
-      ok = (*abort_flag == 0);
-      ptx::tc_fence_after();
-    };
     // this CTA's raw q/k/v tiles of chunk `chunk` (slot chunk % NR)
     auto issue_tma = [&](int chunk) {
       const int s = chunk % NR;
@@ -522,105 +538,82 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::tma_load_3d(rs + RS_QHI, &tm_q, bar, 64, j, t0);
       ptx::tma_load_3d(rs + RS_V, &tm_v, bar, slice * DVS, h, t0);
     };
-    int issued = 0;    // chunks whose tiles have been requested
-    int consumed = 0;  // chunks whose tiles this warpgroup has waited for
+    int issued = 0;    // chunks whose tiles have been requested (thread 64)
+    int consumed = 0;  // chunks whose tiles are known to have landed
     if (t == 64)
       for (; issued < NR && issued < nchunks; ++issued) issue_tma(issued);
-    auto wait_mma = [&]() {
-      wait_bar(bars + BAR_MMAS, ph_mma);
-      ph_mma ^= 1u;
-    };
-    auto publish = [&]() {
-      ptx::fence_proxy_async_smem();
-      ptx::tc_fence_before();
-      named_bar_n(2, 128);
-    };
+    // warps 8-9 own the token rows of U - W S (TMEM lanes 0..63); warps 10-11
+    // the output rows (lanes 64..127).  Per chunk every thread passes the same
+    // barriers whether or not a wait has expired, and all four warps leave the
+    // loop together at the second 128-thread barrier.
+    const bool vrow = t < 64;
 
-    for (int c = 0; c < nchunks && ok; ++c) {
+    for (int c = 0; c < nchunks; ++c) {
       const int rsl = c % NR, psl = c % NP;
-      const int64_t c0t = seq_start + (int64_t)c * C;
+      const uint32_t par = (uint32_t)(c & 1);
       const uint32_t ra = sb + OFF_RAW + rsl * kRaw;
       uint8_t* ps = sm + OFF_PROD + psl * kProd;
       const uint32_t pa = sb + OFF_PROD + psl * kProd;
       const float* spp = sp + psl * SP_N;
-      // this CTA's tiles, then the products (built here or by the other CTA)
-      if (t == 0) {
-        if (!ptx::mbar_wait_bounded(bars + BAR_RAWF + rsl, (uint32_t)((c / NR) & 1), kWaitNs)) *abort_flag = 1;
-        if (!ptx::mbar_wait_cluster_bounded(bars + BAR_PRODF + psl, (uint32_t)((c / NP) & 1), kWaitNs))
-          *abort_flag = 1;
+      const uint32_t tm_qs = TM_QS + 64u * par;  // [K S; Q S] alternates between two column blocks
+      if (vrow) {
+        // U - W S (the products hold -W) and [K S; Q S]
+        if (t == 0) {
+          if (!ptx::mbar_wait_bounded(bars + BAR_RAWF + rsl, (uint32_t)((c / NR) & 1), kWaitNs) ||
+              !ptx::mbar_wait_cluster_bounded(bars + BAR_PRODF + psl, (uint32_t)((c / NP) & 1), kWaitNs))
+            *abort_flag = 1;
+          if (*abort_flag == 0) {
+            ptx::fence_proxy_async_smem();  // products stored by threads (possibly of the other CTA)
+            ptx::tc_fence_after();
+            mma_k64(tmem + TM_U, pa + PS_TU, ra + RS_V, 8192, ID_KMN64, 0);
+            mma_k128(tmem + TM_U, pa + PS_WLO, pa + PS_WHI, sb + OFF_S, 8192, ID_KMN64, 1);
+            ptx::mma_commit(bars + BAR_MMAS);
+            mma_k128(tmem + tm_qs, ra + RS_KLO, ra + RS_KHI, sb + OFF_S, 8192, ID_KMN64, 0);
+            if (!ptx::mbar_wait_bounded(bars + BAR_MMAS, par, kWaitNs)) *abort_flag = 1;
+          }
+        }
+        named_bar_n(3, 64);
+        ok = (*abort_flag == 0);
+        ptx::tc_fence_after();
+        if (ok) {
+          // V' = U - W S and W' = diag(rk exp(g_last - gcum)) V'  (into the W tiles)
+          const float w = spp[SP_WK + t];
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            float u[32];
+            ptx::tmem_ld32(tl + TM_U + 32 * hh, u);
+            ptx::tmem_ld_wait();
+            ptx::st_half_bf16(ps + PS_WLO, t, hh, u);
+#pragma unroll
+            for (int cc = 0; cc < 32; ++cc) u[cc] *= w;
+            ptx::st_half_bf16(ps + PS_WHI, t, hh, u);
+          }
+        }
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_before();
+        named_bar_n(3, 64);
+        if (t == 0 && *abort_flag == 0) {
+          // D4 = K^T W' (the recurrence), then P V' (A = [junk; P]: rows land in
+          // lanes 64..127) once the output warps have read the previous one
+          ptx::tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            ptx::mma_bf16(tmem + TM_D4, mndesc(ra + RS_KLO + 2048 * kk, RS_KHI - RS_KLO),
+                          mndesc(pa + PS_WHI + 2048 * kk, 8192), ID_MNMN64, kk > 0);
+          ptx::mma_commit(bars + BAR_MMAD4);
+          if (c > 0 && !ptx::mbar_wait_bounded(bars + BAR_OUTD, par ^ 1u, kWaitNs)) *abort_flag = 1;
+          ptx::tc_fence_after();
+          mma_k64(tmem + TM_PV, pa + PS_P - kTile, pa + PS_WLO, 8192, ID_KMN64, 0);
+          ptx::mma_commit(bars + BAR_MMAO);
+        }
       }
+      // S <- exp(g_last) S + D4   (thread t owns row t)
+      if (t == 0 && *abort_flag == 0 && !ptx::mbar_wait_bounded(bars + BAR_MMAD4, par, kWaitNs)) *abort_flag = 1;
       named_bar_n(2, 128);
       ok = (*abort_flag == 0);
       ptx::tc_fence_after();
-      if (!ok) break;
-      consumed = c + 1;
-      // [K S; Q S],  W S (A = [W; junk]),  U = T diag(beta) V (A = [Tb; junk])
-      if (t == 0) {
-        ptx::fence_proxy_async_smem();  // products stored by threads (possibly of the other CTA)
-        mma_k128(tmem + TM_KQS, ra + RS_KLO, ra + RS_KHI, sb + OFF_S, 8192, ID_KMN64);
-        mma_k128(tmem + TM_WS, pa + PS_WLO, pa + PS_WHI, sb + OFF_S, 8192, ID_KMN64);
-        mma_k64(tmem + TM_U, pa + PS_TU, ra + RS_V, 8192, ID_KMN64, 0);
-        ptx::mma_commit(bars + BAR_MMAS);
-      }
-      wait_mma();
-      if (!ok) break;
-      if (t < 64) {
-        // V' = U - W S, and W' = diag(rk exp(g_last - gcum)) V'  (into the W tiles)
-        const float w = spp[SP_WK + t];
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          float u[32], ws[32];
-          ptx::tmem_ld32(tl + TM_U + 32 * hh, u);
-          ptx::tmem_ld32(tl + TM_WS + 32 * hh, ws);
-          ptx::tmem_ld_wait();
-#pragma unroll
-          for (int cc = 0; cc < 32; ++cc) u[cc] -= ws[cc];
-          ptx::st_half_bf16(ps + PS_WLO, t, hh, u);
-#pragma unroll
-          for (int cc = 0; cc < 32; ++cc) u[cc] *= w;
-          ptx::st_half_bf16(ps + PS_WHI, t, hh, u);
-        }
-      }
-      publish();
-      // P V' (A = [junk; P]: rows land in lanes 64..127) and D4 = K^T W'
-      if (t == 0) {
-        ptx::tc_fence_after();
-        mma_k64(tmem + TM_PV, pa + PS_P - kTile, pa + PS_WLO, 8192, ID_KMN64, 0);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          ptx::mma_bf16(tmem + TM_D4, mndesc(ra + RS_KLO + 2048 * kk, RS_KHI - RS_KLO),
-                        mndesc(pa + PS_WHI + 2048 * kk, 8192), ID_MNMN64, kk > 0);
-        ptx::mma_commit(bars + BAR_MMAS);
-      }
-      wait_mma();
-      if (!ok) break;
-      if (t >= 64) {
-        // O = diag(exp(gcum) rq) Q S + P V'
-        const int orow = t - 64;
-        const int64_t tok = c0t + orow;
-        const float f = spp[SP_SQ + orow];
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          float qs[32], pv[32];
-          ptx::tmem_ld32(tl + TM_KQS + 32 * hh, qs);
-          ptx::tmem_ld32(tl + TM_PV + 32 * hh, pv);
-          ptx::tmem_ld_wait();
-          if (tok < seq_end) {
-            uint4* op = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + ((size_t)tok * nv + h) * dv +
-                                                 slice * DVS + 32 * hh);
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-              uint4 w;
-              w.x = ptx::pack_bf16x2(fmaf(f, qs[8 * cc + 0], pv[8 * cc + 0]), fmaf(f, qs[8 * cc + 1], pv[8 * cc + 1]));
-              w.y = ptx::pack_bf16x2(fmaf(f, qs[8 * cc + 2], pv[8 * cc + 2]), fmaf(f, qs[8 * cc + 3], pv[8 * cc + 3]));
-              w.z = ptx::pack_bf16x2(fmaf(f, qs[8 * cc + 4], pv[8 * cc + 4]), fmaf(f, qs[8 * cc + 5], pv[8 * cc + 5]));
-              w.w = ptx::pack_bf16x2(fmaf(f, qs[8 * cc + 6], pv[8 * cc + 6]), fmaf(f, qs[8 * cc + 7], pv[8 * cc + 7]));
-              op[cc] = w;
-            }
-          }
-        }
-      }
-      {
+      if (ok) {
+        consumed = c + 1;
         const float decay = spp[SP_GAMMA];
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
@@ -632,16 +625,59 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ptx::st_row_bf16(sm + OFF_S, t, S);
       }
-      publish();
-      if (t == 64) {  // off the polling thread's path
-        // release the product slot to the CTA that builds chunk c + 2
-        if ((c & 1) == (int)crank)
-          ptx::mbar_arrive(bars + BAR_PRODE + psl);
-        else
-          ptx::mbar_arrive_remote(ptx::mapa(ptx::smem_u32(bars + BAR_PEERF + psl), peer));
-        if (c + NR < nchunks) {  // every read of this raw slot has completed
-          issue_tma(c + NR);
-          issued = c + NR + 1;
+      ptx::fence_proxy_async_smem();
+      ptx::tc_fence_before();
+      ok = !named_bar_any(2, 128, *abort_flag != 0);
+      if (!ok) break;
+      if (!vrow) {
+        // output rows, off the recurrence's critical path:
+        // O = diag(exp(gcum) rq) Q S + P V'
+        const int orow = t - 64;
+        const int64_t tok = seq_start + (int64_t)c * C + orow;
+        if (t == 64) {
+          if (c + NR < nchunks) {  // every read of this raw slot has completed (D4 was the last)
+            issue_tma(c + NR);
+            issued = c + NR + 1;
+          }
+          if (!ptx::mbar_wait_bounded(bars + BAR_MMAO, par, kWaitNs)) *abort_flag = 1;
+        }
+        const float f = spp[SP_SQ + orow];  // read before the slot is released below
+        named_bar_n(4, 64);
+        const bool ook = (*abort_flag == 0);
+        ptx::tc_fence_after();
+        if (t == 64) {
+          // release the product slot to the CTA that builds chunk c + 2
+          if ((c & 1) == (int)crank)
+            ptx::mbar_arrive(bars + BAR_PRODE + psl);
+          else
+            ptx::mbar_arrive_remote(ptx::mapa(ptx::smem_u32(bars + BAR_PEERF + psl), peer));
+        }
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+          float qs[16], pv[16];
+          if (ook) {
+            ptx::tmem_ld16(tl + tm_qs + 16 * qq, qs);
+            ptx::tmem_ld16(tl + TM_PV + 16 * qq, pv);
+            ptx::tmem_ld_wait();
+          }
+          if (qq == 3) {  // both accumulators have been read: they may be overwritten
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bars + BAR_OUTD);
+          }
+          if (ook && tok < seq_end) {
+            uint4* op = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + ((size_t)tok * nv + h) * dv +
+                                                 slice * DVS + 16 * qq);
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+              uint4 w;
+              w.x = ptx::pack_bf16x2(fmaf(f, qs[8 * cc + 0], pv[8 * cc + 0]), fmaf(f, qs[8 * cc + 1], pv[8 * cc + 1]));
+              w.y = ptx::pack_bf16x2(fmaf(f, qs[8 * cc + 2], pv[8 * cc + 2]), fmaf(f, qs[8 * cc + 3], pv[8 * cc + 3]));
+              w.z = ptx::pack_bf16x2(fmaf(f, qs[8 * cc + 4], pv[8 * cc + 4]), fmaf(f, qs[8 * cc + 5], pv[8 * cc + 5]));
+              w.w = ptx::pack_bf16x2(fmaf(f, qs[8 * cc + 6], pv[8 * cc + 6]), fmaf(f, qs[8 * cc + 7], pv[8 * cc + 7]));
+              op[cc] = w;
+            }
+          }
         }
       }
     }

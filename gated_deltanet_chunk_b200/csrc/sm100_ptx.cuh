@@ -123,6 +123,25 @@ __device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t* bar, uint32_
     if (globaltimer_ns() - t0 > limit_ns) return false;
   }
 }
+// Asynchronous 16-byte / 4-byte stores into another CTA's shared memory; each
+// completes `bytes` of transaction count on the mbarrier `cluster_bar` there.
+__device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, uint4 v, uint32_t cluster_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                   cluster_addr),
+               "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(cluster_bar)
+               : "memory");
+}
+__device__ __forceinline__ void st_async_b32(uint32_t cluster_addr, uint32_t v, uint32_t cluster_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(cluster_addr),
+               "r"(v), "r"(cluster_bar)
+               : "memory");
+}
+// arrive on another CTA's mbarrier announcing `bytes` of incoming transactions
+__device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t cluster_bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(cluster_bar),
+               "r"(bytes)
+               : "memory");
+}
 __device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
@@ -197,6 +216,16 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
         "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
 }
+// 16 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // ------------------------------------------------------------------ descriptors
@@ -264,24 +293,27 @@ __device__ __forceinline__ uint4 pack8_bf16(const float* v) {
   return w;
 }
 
-// Like st_half_bf16 / st_row_bf16, also storing the same bytes to `remote`,
-// the shared::cluster address of the same tile in another CTA of the cluster.
-__device__ __forceinline__ void st_half_bf16_dual(uint8_t* tile, uint32_t remote, int r, int half, const float* v) {
+// Like st_half_bf16 / st_row_bf16, also sending the same bytes with st.async
+// to `remote`, the shared::cluster address of the same tile in another CTA of
+// the cluster, completing transactions on that CTA's mbarrier `rbar`.
+__device__ __forceinline__ void st_half_bf16_dual(uint8_t* tile, uint32_t remote, uint32_t rbar, int r, int half,
+                                                  const float* v) {
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
     const uint4 w = pack8_bf16(v + 8 * c);
     const uint32_t off = sw128_off(r, 4 * half + c);
     *reinterpret_cast<uint4*>(tile + off) = w;
-    st_cluster_v4(remote + off, w);
+    st_async_v4(remote + off, w, rbar);
   }
 }
-__device__ __forceinline__ void st_row_bf16_dual(uint8_t* tile, uint32_t remote, int r, const float* v) {
+__device__ __forceinline__ void st_row_bf16_dual(uint8_t* tile, uint32_t remote, uint32_t rbar, int r,
+                                                 const float* v) {
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
     const uint4 w = pack8_bf16(v + 8 * c);
     const uint32_t off = sw128_off(r, c);
     *reinterpret_cast<uint4*>(tile + off) = w;
-    st_cluster_v4(remote + off, w);
+    st_async_v4(remote + off, w, rbar);
   }
 }
 
