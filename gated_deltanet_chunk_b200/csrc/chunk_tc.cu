@@ -5,34 +5,36 @@
 // columns.  The two CTAs of a (sequence, v-head) form a cluster.  In each CTA:
 //
 //   intra warps (0-7): the state-independent part of a chunk -- gate cumsum,
-//     L2 norms, G = [K;Q] K^T, the A and P matrices, T = (I - A)^-1 and W.
+//     L2 norms, G = [K;Q] K^T, the A and P matrices and T = (I - A)^-1.
 //     Chunk c is built only by cluster rank c % 2, which writes the products
-//     (W, P, T diag(beta), per-row scalars) into its own product slot and,
-//     with st.async into distributed shared memory, into the same slot of the
-//     other CTA, whose mbarrier completes when all those bytes have landed.
+//     (-T diag(bw), P, T diag(beta), per-row scalars) into its own product slot
+//     and, with st.async into distributed shared memory, into the same slot of
+//     the other CTA, whose mbarrier completes when all those bytes have landed.
 //     Each CTA thus builds every other chunk for both Dv slices.
 //   serial warps (8-11): the state recurrence for this CTA's Dv slice.  The
 //     fp32 state slice S [128 x 64] lives in registers (thread d holds row d)
 //     and, rounded to bf16, in shared memory as the B operand of the next
 //     chunk.  The critical path per chunk is two tensor-core round trips
-//     (U - W S, then D4) and two short epilogues; the output rows (P V' + Q S)
-//     are finished by warps 10-11 while warps 8-9 start the next chunk.  The
-//     serial warps also refill this CTA's 3-deep TMA ring of raw q/k/v tiles.
+//     (V', then D4) and two short epilogues; -W is formed before S is needed,
+//     and the output rows (P V' + Q S) are finished by warps 10-11 while
+//     warps 8-9 start the next chunk.  The serial warps also refill this CTA's
+//     3-deep TMA ring of raw q/k/v tiles.
 //
 // Algebra: the chunkwise form of the "手撕Qwen3-Next" walkthrough, section
 // 一(一)5(1), steps c-f, with the L2 norms folded into row scales
 // (rk = 1/|k|, rq = scale/|q|) so the raw TMA-loaded q/k tiles are the MMA
 // operands.  Gamma[r][i] = exp(gcum_r - gcum_i) is formed only for i <= r
-// (mask before exp), once per chunk, as the table GK[r][i] = rk_i Gamma[r][i].
+// (mask before exp), on the fly while G is scaled.
 //   G  = [K; Q] K^T                                     tcgen05 M=128 N=64 K=128
-//   A  = -strictLower(diag(beta rk) (K K^T) * GK)                      CUDA cores
-//   P  = diag(rq) (Q K^T) * GK  (lower incl. diagonal)                  CUDA cores
+//   A  = -strictLower(diag(beta rk) (K K^T) diag(rk) * Gamma)          CUDA cores
+//   P  = diag(rq) (Q K^T) diag(rk) * Gamma  (lower incl. diagonal)      CUDA cores
 //   T  = (I - A)^-1 = R + N^2 R,  R = T_D + N T_D,  N = T_D A_off       3 tcgen05 rounds
-//        (T_D: inverse of A's 16x16 diagonal blocks by forward substitution
-//        in registers; A_off: the strictly block-lower part of A; N^4 = 0.
-//        The 16-row block scheme is the PyPTO README's inverse_pto submodule.)
-//   W  = T diag(beta exp(gcum) rk) K  (stored negated)                  tcgen05
-//   serial:  V' = T diag(beta) V + (-W) S   (one accumulator)           one round
+//        (T_D: inverse of A's 16x16 diagonal blocks, one column per lane by
+//        forward substitution; A_off: the strictly block-lower part of A;
+//        N^4 = 0.  The 16-row block scheme is the PyPTO README's inverse_pto
+//        submodule.)
+//   serial:  -W = (-T diag(beta exp(gcum) rk)) K                        one round
+//            V' = T diag(beta) V + (-W) S   (one accumulator)           one round
 //            [KS; QS] = [K; Q] S                                  same round, own use
 //            D4 = K^T diag(rk exp(g_last - gcum)) V'                    one round
 //            PV = P V'                                            after D4, own use
@@ -70,29 +72,34 @@ constexpr int kTile = 64 * 128;  // 64 rows x 128 bytes (64 bf16)
 // raw slot: [K_lo | Q_lo] [K_hi | Q_hi] V
 constexpr int RS_KLO = 0, RS_QLO = 1 * kTile, RS_KHI = 2 * kTile, RS_QHI = 3 * kTile, RS_V = 4 * kTile;
 constexpr int kRaw = 5 * kTile;
-// product slot: [W_lo | W_hi | P | T diag(beta)]; W_lo/W_hi hold V' / W' once
-// the serial side has read W.
+// product slot: [W_lo | W_hi | P | T diag(beta)].  The builder stores
+// -T diag(bw) in W_hi; the serial side forms -W = (-T diag(bw)) K from it into
+// W_lo / W_hi, and later overwrites those with V' / W'.
 constexpr int PS_WLO = 0, PS_WHI = 1 * kTile, PS_P = 2 * kTile, PS_TU = 3 * kTile;
 constexpr int kProd = 4 * kTile;
 constexpr int OFF_RAW = 0;
 constexpr int OFF_PROD = NR * kRaw;
-constexpr int OFF_X0 = OFF_PROD + NP * kProd;  // intra scratch: GK table (X0+X1), A_off, N, N^2, T diag(bw)
+constexpr int OFF_X0 = OFF_PROD + NP * kProd;  // intra scratch: A_off, N, N^2
 constexpr int OFF_X1 = OFF_X0 + kTile;         // intra scratch: T_D, R
 constexpr int OFF_S = OFF_X1 + kTile;          // serial: S operand, 128 rows (d) x 64 cols
 constexpr int OFF_SCI = OFF_S + 2 * kTile;     // intra scalars
 constexpr int SI_RK = 0, SI_RQ = 64, SI_BETA = 128, SI_GC = 192, SI_BW = 256, SI_NP = 320, SI_WK = 576,
-              SI_SQ = 640, SI_GAM = 704, SI_N = 708;
-constexpr int OFF_SCP = OFF_SCI + SI_N * 4;    // per-product-slot scalars for the serial side
+              SI_SQ = 640, SI_GAM = 704, SI_CF = 708, SI_N = 772;
+// diagonal 16 x 16 blocks of A, then of T_D, as fp32 (4 blocks, padded so the
+// two blocks a warp handles sit in different banks)
+constexpr int LS_BLK = 16 * 16 + 16;
+constexpr int OFF_LS = OFF_SCI + SI_N * 4;
+constexpr int OFF_SCP = OFF_LS + 4 * LS_BLK * 4;  // per-product-slot scalars for the serial side
 constexpr int SP_WK = 0, SP_SQ = 64, SP_GAMMA = 128, SP_N = 132;
-// bytes one CTA sends to the other per chunk it builds: W, P, T diag(beta), wk, sq, gamma
-constexpr uint32_t kPushBytes = 4 * 8192 + (2 * 64 + 1) * 4;
+// bytes one CTA sends to the other per chunk it builds: -T diag(bw), P, T diag(beta), wk, sq, gamma
+constexpr uint32_t kPushBytes = 3 * 8192 + (2 * 64 + 1) * 4;
 constexpr int OFF_BAR = OFF_SCP + NP * SP_N * 4;
 // barriers: raw_full[NR]; prod_full[NP] (the products of a chunk have landed in
 // this CTA); prod_free[NP] (this CTA's serial warps are done with the slot);
 // peer_free[NP] (the other CTA's serial warps are done with its copy); mma_i, mma_s
 constexpr int BAR_RAWF = 0, BAR_PRODF = NR, BAR_PRODE = NR + NP, BAR_PEERF = NR + 2 * NP;
 constexpr int BAR_MMAI = NR + 3 * NP, BAR_MMAS = BAR_MMAI + 1, BAR_MMAD4 = BAR_MMAS + 1, BAR_MMAO = BAR_MMAD4 + 1;
-constexpr int BAR_OUTD = BAR_MMAO + 1, NBAR = BAR_OUTD + 1;
+constexpr int BAR_OUTD = BAR_MMAO + 1, BAR_MMAW = BAR_OUTD + 1, NBAR = BAR_MMAW + 1;
 constexpr int SMEM_USED = OFF_BAR + NBAR * 8 + 16;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
 static_assert(OFF_BAR % 8 == 0, "mbarrier alignment");
@@ -100,11 +107,12 @@ static_assert(SMEM_BYTES <= 232448, "shared memory");
 
 // ---- TMEM columns (128 lanes x 512 fp32 columns)
 constexpr uint32_t TM_G = 0;     // intra: G; then N; then N^2 R
-constexpr uint32_t TM_N2 = 64;   // intra: [N^2 | N T_D] (128 cols); then W (128 cols)
+constexpr uint32_t TM_N2 = 64;   // intra: [N^2 | N T_D] (128 cols)
 constexpr uint32_t TM_QS = 192;  // serial: [K S ; Q S], two column blocks used alternately (128 cols)
+constexpr uint32_t TM_W = 320;   // serial: -W (128 cols: the U and D4 blocks, both free at that point)
 constexpr uint32_t TM_U = 320;   // serial: U - W S (rows 0..63)
-constexpr uint32_t TM_PV = 384;  // serial: P V' (rows 64..127)
-constexpr uint32_t TM_D4 = 448;  // serial: state update
+constexpr uint32_t TM_D4 = 384;  // serial: state update
+constexpr uint32_t TM_PV = 448;  // serial: P V' (rows 64..127)
 constexpr uint32_t TM_COLS = 512;
 
 constexpr uint32_t ID_KK64 = ptx::idesc_bf16_f32(128, 64, false, false);
@@ -112,7 +120,9 @@ constexpr uint32_t ID_KMN64 = ptx::idesc_bf16_f32(128, 64, false, true);
 constexpr uint32_t ID_KMN128 = ptx::idesc_bf16_f32(128, 128, false, true);
 constexpr uint32_t ID_MNMN64 = ptx::idesc_bf16_f32(128, 64, true, true);
 
-__device__ __forceinline__ float fast_exp(float x) { return __expf(x); }
+// exp(x) as 2^(x log2 e) on the special-function unit, flushing results below
+// the fp32 normal range to zero (such decay factors contribute nothing here)
+__device__ __forceinline__ float fast_exp(float x) { return ptx::ex2_approx(x * 1.4426950408889634f); }
 __device__ __forceinline__ uint64_t kdesc(uint32_t addr) { return ptx::sdesc_sw128(addr, 16, 1024); }
 __device__ __forceinline__ uint64_t mndesc(uint32_t addr, uint32_t lbo) { return ptx::sdesc_sw128(addr, lbo, 1024); }
 
@@ -159,9 +169,6 @@ __device__ __forceinline__ bool named_bar_any(int id, int nthreads, bool flag) {
   return r != 0;
 }
 
-// GK table: fp32 [64][64], rows of 256 bytes with the 16-byte chunk k of row r
-// stored at chunk position k ^ (r & 7) (conflict-free row reads).
-__device__ __forceinline__ int gk_index(int r, int i) { return r * 64 + ((((i >> 2) ^ (r & 7))) << 2) + (i & 3); }
 
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -200,6 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::mbar_init(bars + BAR_MMAD4, 1);
     ptx::mbar_init(bars + BAR_MMAO, 1);
     ptx::mbar_init(bars + BAR_OUTD, 2);
+    ptx::mbar_init(bars + BAR_MMAW, 1);
     *abort_flag = 0;
     ptx::fence_mbar_init();
     ptx::prefetch_tensormap(&tm_q);
@@ -277,7 +285,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint8_t* ps = sm + OFF_PROD + psl * kProd;
       const uint32_t pa = sb + OFF_PROD + psl * kProd;
       float* spp = sp + psl * SP_N;
-      float* gk = reinterpret_cast<float*>(sm + OFF_X0);  // 16 KB: the X0 / X1 scratch tiles
       const uint32_t rpa = ptx::mapa(pa, peer);                     // the other CTA's copy of the slot
       const uint32_t rspp = ptx::mapa(ptx::smem_u32(spp), peer);
       const uint32_t rbar = ptx::mapa(ptx::smem_u32(bars + BAR_PRODF + psl), peer);  // the other CTA's prod_full
@@ -333,56 +340,98 @@ __global__ void __launch_bounds__(kThreads, 1)
         si[(t < 64 ? SI_RK : SI_RQ) + nr] = valid ? f : 0.f;
       }
       named_bar_n(1, 256);
-      // GK[r][i] = rk_i exp(gcum_r - gcum_i) for i <= r (else 0); row scalars
-#pragma unroll 4
-      for (int e = t; e < 64 * 64; e += 256) {
-        const int gr = e >> 6, gi = e & 63;
-        const float val = (gi <= gr) ? si[SI_RK + gi] * fast_exp(si[SI_GC + gr] - si[SI_GC + gi]) : 0.f;
-        gk[gk_index(gr, gi)] = val;
-      }
+      // row scalars; CF_i = rk_i exp(gcum_b - gcum_i) with b = the last column
+      // of i's 32-column half (the pivot for rows below that half)
       if (t < 64) {
         const float gl = si[SI_GC + 63], gr = si[SI_GC + t];
         const float eg = fast_exp(gr);
         const float rk = si[SI_RK + t];
+        si[SI_CF + t] = rk * fast_exp(si[SI_GC + (t | 31)] - gr);
         si[SI_BW + t] = si[SI_BETA + t] * eg * rk;
         si[SI_WK + t] = rk * fast_exp(gl - gr);
         si[SI_SQ + t] = eg * si[SI_RQ + t];
         if (t == 0) si[SI_GAM] = fast_exp(gl);
       }
-      wait_mma();  // G ready (the named barrier inside also publishes GK)
+      wait_mma();  // G ready (the named barrier inside also publishes the scalars)
       if (!ok) break;
       // A rows (key rows) with the diagonal-block inverse; P rows (query rows)
       float keep[32];  // key rows: R = T_D + N T_D (this half); query rows: this half of P
       float t16[16];   // diagonal-block threads: strictly lower part of this row's T_D block
       {
+        // G row r, columns [c0, c0 + 32), scaled to A (key rows) or P (query rows):
+        //   A[r][i] = -beta_r rk_r rk_i exp(gcum_r - gcum_i) (K K^T)[r][i],  i < r
+        //   P[r][i] =  rq_r rk_i exp(gcum_r - gcum_i) (Q K^T)[r][i],        i <= r
+        // The decay is formed only where i <= r (mask before exp).  In a half that
+        // lies wholly below row r it is split at the half's last column b,
+        // exp(gcum_r - gcum_b) exp(gcum_b - gcum_i), both factors <= 1 for gates <= 0.
         float av[32];
         ptx::tmem_ld32(tl + TM_G + c0, av);
         ptx::tmem_ld_wait();
         const float f = krow ? -si[SI_BETA + r] * si[SI_RK + r] : si[SI_RQ + r];
-        const float4* gkr = reinterpret_cast<const float4*>(gk + r * 64);
+        const int rblk = r >> 5;  // == q & 1: warp-uniform
+        if (rblk > hf) {
+          const float rowf = f * fast_exp(si[SI_GC + r] - si[SI_GC + c0 + 31]);
+          const float4* cf = reinterpret_cast<const float4*>(si + SI_CF + c0);
 #pragma unroll
-        for (int k4 = 0; k4 < 8; ++k4) {
-          const float4 x = gkr[(8 * hf + k4) ^ (r & 7)];
-          av[4 * k4 + 0] *= f * x.x;
-          av[4 * k4 + 1] *= f * x.y;
-          av[4 * k4 + 2] *= f * x.z;
-          av[4 * k4 + 3] *= f * x.w;
+          for (int k4 = 0; k4 < 8; ++k4) {
+            const float4 x = cf[k4];
+            av[4 * k4 + 0] *= rowf * x.x;
+            av[4 * k4 + 1] *= rowf * x.y;
+            av[4 * k4 + 2] *= rowf * x.z;
+            av[4 * k4 + 3] *= rowf * x.w;
+          }
+        } else if (rblk == hf) {
+          const float gr = si[SI_GC + r];
+          const int lim = krow ? r : r + 1;  // columns i < lim are kept
+          const float4* rk4 = reinterpret_cast<const float4*>(si + SI_RK + c0);
+          const float4* gc4 = reinterpret_cast<const float4*>(si + SI_GC + c0);
+#pragma unroll
+          for (int k4 = 0; k4 < 8; ++k4) {
+            const float4 rk = rk4[k4], gc = gc4[k4];
+            const int i0 = c0 + 4 * k4;
+            av[4 * k4 + 0] = (i0 + 0 < lim) ? av[4 * k4 + 0] * (f * rk.x) * fast_exp(gr - gc.x) : 0.f;
+            av[4 * k4 + 1] = (i0 + 1 < lim) ? av[4 * k4 + 1] * (f * rk.y) * fast_exp(gr - gc.y) : 0.f;
+            av[4 * k4 + 2] = (i0 + 2 < lim) ? av[4 * k4 + 2] * (f * rk.z) * fast_exp(gr - gc.z) : 0.f;
+            av[4 * k4 + 3] = (i0 + 3 < lim) ? av[4 * k4 + 3] * (f * rk.w) * fast_exp(gr - gc.w) : 0.f;
+          }
+        } else {
+#pragma unroll
+          for (int cc = 0; cc < 32; ++cc) av[cc] = 0.f;
         }
-        named_bar_n(1, 256);  // every GK row has been read: X0 / X1 are free
         if (krow) {
-#pragma unroll
-          for (int cc = 0; cc < 32; ++cc) av[cc] = (c0 + cc == r) ? 0.f : av[cc];  // strictly lower
           if (diag_here) {
+            // T_D = (I - A_D)^-1 for this warp's two 16 x 16 diagonal blocks
+            // (lanes 0-15: block 2 rblk, lanes 16-31: block 2 rblk + 1).  Lane li
+            // first publishes row li of A_D column-major, then solves column li of
+            // T_D = I + A_D T_D top to bottom, then reads back row li of T_D.
+            float* ls = reinterpret_cast<float*>(sm + OFF_LS) + (2 * rblk + (lane >> 4)) * LS_BLK;
 #pragma unroll
-            for (int jj = 0; jj < 16; ++jj) t16[jj] = lane < 16 ? av[jj] : av[16 + jj];
+            for (int k = 0; k < 16; ++k) ls[k * 16 + li] = lane < 16 ? av[k] : av[16 + k];  // A_D[li][k] (0 for k >= li)
+            __syncwarp();
+            float x[16];
 #pragma unroll
-            for (int m = 1; m < 15; ++m) {
-              const float coef = t16[m];
+            for (int i = 0; i < 16; ++i) x[i] = (i == li) ? 1.f : 0.f;
 #pragma unroll
-              for (int jj = 0; jj < m; ++jj) {
-                const float bj = __shfl_sync(0xffffffffu, t16[jj], (lane & 16) | m);
-                if (li > m) t16[jj] = fmaf(coef, bj, t16[jj]);
+            for (int k = 0; k < 15; ++k) {
+              float colk[16];
+              const float4* c4 = reinterpret_cast<const float4*>(ls + k * 16);
+#pragma unroll
+              for (int v = 0; v < 4; ++v) {
+                const float4 y = c4[v];
+                colk[4 * v] = y.x; colk[4 * v + 1] = y.y; colk[4 * v + 2] = y.z; colk[4 * v + 3] = y.w;
               }
+#pragma unroll
+              for (int i = k + 1; i < 16; ++i) x[i] = fmaf(colk[i], x[k], x[i]);
+            }
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) ls[i * 16 + li] = x[i];  // T_D[i][li], now row-major
+            __syncwarp();
+            const float4* r4 = reinterpret_cast<const float4*>(ls + li * 16);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const float4 y = r4[v];
+              t16[4 * v] = y.x; t16[4 * v + 1] = y.y; t16[4 * v + 2] = y.z; t16[4 * v + 3] = y.w;
             }
           }
           td_half(t16, keep);
@@ -454,51 +503,46 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = !named_bar_any(1, 256, *abort_flag != 0);
       ptx::tc_fence_after();
       if (!ok) break;
+      // products: stored locally first (and made visible to this CTA's tensor
+      // cores), then sent to the other CTA with st.async
+      uint4 pk0[4], pk1[4];
       if (t < 64) {
-        const float wk = si[SI_WK + t], sq = si[SI_SQ + t];
-        spp[SP_WK + t] = wk;
-        spp[SP_SQ + t] = sq;
-        ptx::st_async_b32(rspp + 4 * (SP_WK + t), __float_as_uint(wk), rbar);
-        ptx::st_async_b32(rspp + 4 * (SP_SQ + t), __float_as_uint(sq), rbar);
-        if (t == 0) {
-          spp[SP_GAMMA] = si[SI_GAM];
-          ptx::st_async_b32(rspp + 4 * SP_GAMMA, __float_as_uint(si[SI_GAM]), rbar);
-        }
+        spp[SP_WK + t] = si[SI_WK + t];
+        spp[SP_SQ + t] = si[SI_SQ + t];
+        if (t == 0) spp[SP_GAMMA] = si[SI_GAM];
       }
-      if (!krow) ptx::st_half_bf16_dual(ps + PS_P, rpa + PS_P, rbar, r, hf, keep);  // P
-      if (krow) {
+      if (!krow) {
+        ptx::pack_half_bf16(keep, pk0);  // P
+        ptx::st_half_packed(ps + PS_P, r, hf, pk0);
+      } else {
         float x[32];
         ptx::tmem_ld32(tl + TM_G + c0, x);
         ptx::tmem_ld_wait();
 #pragma unroll
         for (int cc = 0; cc < 32; ++cc) x[cc] += keep[cc];  // T = R + N^2 R
 #pragma unroll
-        for (int cc = 0; cc < 32; ++cc) keep[cc] = x[cc] * si[SI_BW + c0 + cc];
-        ptx::st_half_bf16(sm + OFF_X0, r, hf, keep);  // T diag(beta exp(gcum) rk)
+        for (int cc = 0; cc < 32; ++cc) keep[cc] = -x[cc] * si[SI_BW + c0 + cc];
+        ptx::pack_half_bf16(keep, pk0);  // -T diag(beta exp(gcum) rk), for W
+        ptx::st_half_packed(ps + PS_WHI, r, hf, pk0);
 #pragma unroll
         for (int cc = 0; cc < 32; ++cc) keep[cc] = x[cc] * si[SI_BETA + c0 + cc];
-        ptx::st_half_bf16_dual(ps + PS_TU, rpa + PS_TU, rbar, r, hf, keep);  // T diag(beta), for U
+        ptx::pack_half_bf16(keep, pk1);  // T diag(beta), for U
+        ptx::st_half_packed(ps + PS_TU, r, hf, pk1);
       }
-      publish();
-      // W = T diag(bw) K   (A = [T diag(bw); junk])
-      if (t == 0) {
-        ptx::tc_fence_after();
-        mma_k64(tmem + TM_N2, sb + OFF_X0, ra + RS_KLO, RS_KHI - RS_KLO, ID_KMN128, 0);
-        ptx::mma_commit(bars + BAR_MMAI);
+      ptx::fence_proxy_async_smem();
+      if (t < 64) {
+        ptx::st_async_b32(rspp + 4 * (SP_WK + t), __float_as_uint(si[SI_WK + t]), rbar);
+        ptx::st_async_b32(rspp + 4 * (SP_SQ + t), __float_as_uint(si[SI_SQ + t]), rbar);
+        if (t == 0) ptx::st_async_b32(rspp + 4 * SP_GAMMA, __float_as_uint(si[SI_GAM]), rbar);
       }
-      wait_mma();
-      if (!ok) break;
-      if (krow) {
-        // W has 128 columns: this thread writes columns [64 hf, 64 hf + 64)
-        float x[64];
-        ptx::tmem_ld32(tl + TM_N2 + 64 * hf, x);
-        ptx::tmem_ld32(tl + TM_N2 + 64 * hf + 32, x + 32);
-        ptx::tmem_ld_wait();
-#pragma unroll
-        for (int cc = 0; cc < 64; ++cc) x[cc] = -x[cc];  // the serial side accumulates U + (-W) S
-        ptx::st_row_bf16_dual(ps + (hf ? PS_WHI : PS_WLO), rpa + (hf ? PS_WHI : PS_WLO), rbar, r, x);
+      if (!krow) {
+        ptx::st_half_packed_remote(rpa + PS_P, rbar, r, hf, pk0);
+      } else {
+        ptx::st_half_packed_remote(rpa + PS_WHI, rbar, r, hf, pk0);
+        ptx::st_half_packed_remote(rpa + PS_TU, rbar, r, hf, pk1);
       }
-      publish();
+      ptx::tc_fence_before();
+      named_bar_n(1, 256);
       if (t == 0) ptx::mbar_arrive(bars + BAR_PRODF + psl);  // the other CTA's copy completes by transactions
     }
     if (!ok && t == 0) atomicOr(&g_status, 1u);
@@ -557,13 +601,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float* spp = sp + psl * SP_N;
       const uint32_t tm_qs = TM_QS + 64u * par;  // [K S; Q S] alternates between two column blocks
       if (vrow) {
-        // U - W S (the products hold -W) and [K S; Q S]
+        // -W = (-T diag(bw)) K   (A = [-T diag(bw); junk])
         if (t == 0) {
           if (!ptx::mbar_wait_bounded(bars + BAR_RAWF + rsl, (uint32_t)((c / NR) & 1), kWaitNs) ||
               !ptx::mbar_wait_cluster_bounded(bars + BAR_PRODF + psl, (uint32_t)((c / NP) & 1), kWaitNs))
             *abort_flag = 1;
           if (*abort_flag == 0) {
             ptx::fence_proxy_async_smem();  // products stored by threads (possibly of the other CTA)
+            ptx::tc_fence_after();
+            mma_k64(tmem + TM_W, pa + PS_WHI, ra + RS_KLO, RS_KHI - RS_KLO, ID_KMN128, 0);
+            ptx::mma_commit(bars + BAR_MMAW);
+            if (!ptx::mbar_wait_bounded(bars + BAR_MMAW, par, kWaitNs)) *abort_flag = 1;
+          }
+        }
+        named_bar_n(3, 64);
+        ok = (*abort_flag == 0);
+        ptx::tc_fence_after();
+        if (ok) {
+#pragma unroll
+          for (int qq = 0; qq < 4; ++qq) {  // row t of -W, 32 columns at a time, into W_lo | W_hi
+            float x[32];
+            ptx::tmem_ld32(tl + TM_W + 32 * qq, x);
+            ptx::tmem_ld_wait();
+            ptx::st_half_bf16(ps + (qq < 2 ? PS_WLO : PS_WHI), t, qq & 1, x);
+          }
+        }
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_before();
+        named_bar_n(3, 64);
+        // U - W S and [K S; Q S]
+        if (t == 0) {
+          if (*abort_flag == 0) {
             ptx::tc_fence_after();
             mma_k64(tmem + TM_U, pa + PS_TU, ra + RS_V, 8192, ID_KMN64, 0);
             mma_k128(tmem + TM_U, pa + PS_WLO, pa + PS_WHI, sb + OFF_S, 8192, ID_KMN64, 1);

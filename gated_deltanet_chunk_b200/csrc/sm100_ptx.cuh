@@ -76,6 +76,13 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
+// 2^x with flush-to-zero (hardware approximation, relative error ~2^-22)
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // ------------------------------------------------------------------ clusters / DSMEM
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
@@ -291,6 +298,23 @@ __device__ __forceinline__ uint4 pack8_bf16(const float* v) {
   w.z = pack_bf16x2(v[4], v[5]);
   w.w = pack_bf16x2(v[6], v[7]);
   return w;
+}
+
+// A half row (32 fp32 values) packed to four 16-byte bf16 chunks, stored to a
+// local SW128 tile, and sent with st.async to the same place in another CTA's
+// tile (completing transactions on that CTA's mbarrier `rbar`).
+__device__ __forceinline__ void pack_half_bf16(const float* v, uint4* w) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) w[c] = pack8_bf16(v + 8 * c);
+}
+__device__ __forceinline__ void st_half_packed(uint8_t* tile, int r, int half, const uint4* w) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(tile + sw128_off(r, 4 * half + c)) = w[c];
+}
+__device__ __forceinline__ void st_half_packed_remote(uint32_t remote, uint32_t rbar, int r, int half,
+                                                      const uint4* w) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) st_async_v4(remote + sw128_off(r, 4 * half + c), w[c], rbar);
 }
 
 // Like st_half_bf16 / st_row_bf16, also sending the same bytes with st.async
