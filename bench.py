@@ -52,6 +52,34 @@ def decode_bytes(n, nqk, nv, dk, dv, esz):
     return n * nv * dk * dv * 4 * 2 + n * (2 * nqk * dk + 2 * nv * dv) * esz + n * nv * 4 * 2
 
 
+# DRAM traffic per launch from an ncu capture (profiles/traffic.json), valid
+# only while the kernel's sources hash to the value recorded with it.
+KERNEL_SOURCES = {
+    "chunk_fwd_tc": ["chunk_tc.cu", "sm100_ptx.cuh", "gdn_common.cuh"],
+    "recurrent_step": ["decode_step.cu", "gdn_common.cuh"],
+}
+
+
+def source_hash(kernel):
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "gated_deltanet_chunk_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(kernel, units):
+    """Bytes per launch for `units` (tokens or sequences), or None if no capture matches the sources."""
+    try:
+        rec = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))[kernel]
+    except Exception:
+        return None
+    if rec.get("source_sha256") != source_hash(kernel):
+        return None
+    return rec["bytes_per_unit"] * units
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -186,7 +214,7 @@ def run_ours(args, world, rank, local):
 
     def step():
         gdn.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], None, None, chunk_size=C,
-                      out=out, final_state=sf, num_seqs=n)
+                      out=out, final_state=sf, num_seqs=n, kernel=args.kernel)
 
     for _ in range(args.warmup):
         step()
@@ -228,7 +256,8 @@ def run_ours(args, world, rank, local):
                    "parallelism": "replicas x%d" % world},
         "gpu_launches": args.steps,
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks[peak_key],
-                     "unit": "GB/s", "frac": achieved_gbs / peaks[peak_key], "traffic": None,
+                     "unit": "GB/s", "frac": achieved_gbs / peaks[peak_key],
+                     "traffic": recorded_traffic("chunk_fwd_tc", T),
                      "peak_source": peak_src, "alg_bytes_per_launch": bytes_alg,
                      "kernel_ms": kern_ms,
                      "tensor_tflops_tri": fl_tri / (kern_ms / 1e3) / 1e12,
@@ -273,12 +302,13 @@ def run_ours(args, world, rank, local):
         res["decode"] = run_decode(args, world, rank, dev, stream, peaks, peak_src)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
-        tok, dt = time_oracle(host, args.cpu_sample_tokens)
+        t_sample = args.cpu_sample_tokens or T // n
+        tok, dt = time_oracle(host, t_sample)
         res["cpu_baseline"] = {"value": tok / dt, "unit": "tokens/s", "cores": oracle.num_threads(),
                                "kind": "oracle",
                                "sample": "fp64 token loop over the first %d tokens of each of the %d "
                                          "sequences, all %d v-heads (%.1f s wall)"
-                                         % (args.cpu_sample_tokens, n, nv, dt)}
+                                         % (t_sample, n, nv, dt)}
     return res
 
 
@@ -314,7 +344,8 @@ def run_decode(args, world, rank, dev, stream, peaks, peak_src):
     return {"value": wl.num_seqs * steps * world / (ms / 1e3), "unit": "tokens/s",
             "workload": DECODE, "steps": steps, "ms_per_step": per_step_ms, "gpu_launches": steps,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": gbs / peaks["hbm_gbs"], "traffic": None, "peak_source": peak_src,
+                         "frac": gbs / peaks["hbm_gbs"], "traffic": recorded_traffic("recurrent_step", wl.num_seqs),
+                         "peak_source": peak_src,
                          "alg_bytes_per_launch": byts}}
 
 
@@ -360,9 +391,12 @@ def main():
                     help="override the prefill sequence length (profiling of smaller cases)")
     ap.add_argument("--decode-steps", type=int, default=0,
                     help="override the number of decode steps (profiling of smaller cases)")
+    ap.add_argument("--kernel", choices=["auto", "simt", "tc"], default="auto",
+                    help="prefill kernel selection passed to gdn_chunk_fwd (default: auto)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-sample-tokens", type=int, default=4096)
+    ap.add_argument("--cpu-sample-tokens", type=int, default=0,
+                    help="oracle sample per sequence for cpu_baseline (default: the whole workload)")
     ap.add_argument("--ref-sample-tokens", type=int, default=512)
     args = ap.parse_args()
     if args.warmup < 3:
