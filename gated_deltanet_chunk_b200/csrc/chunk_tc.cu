@@ -5,15 +5,16 @@
 // columns.  The two CTAs of a (sequence, v-head) form a cluster.  In each CTA:
 //
 //   intra warps (0-7): the state-independent part of a chunk -- gate cumsum,
-//     L2 norms, G = [K;Q] K^T, the A and P matrices and T = (I - A)^-1.
+//     L2 norms, G = [K;Q] K^T, the A and P matrices and T = (I - A)^-1 (fp32,
+//     CUDA cores).
 //     Chunk c is built only by cluster rank c % 2, which writes the products
 //     (-T diag(bw), P, T diag(beta), per-row scalars) into its own product slot
 //     and, with st.async into distributed shared memory, into the same slot of
 //     the other CTA, whose mbarrier completes when all those bytes have landed.
 //     Each CTA thus builds every other chunk for both Dv slices.
 //   serial warps (8-11): the state recurrence for this CTA's Dv slice.  The
-//     fp32 state slice S [128 x 64] lives in registers (thread d holds row d)
-//     and, rounded to bf16, in shared memory as the B operand of the next
+//     fp32 state slice S [128 x 64] lives in TMEM (lane d holds row d) and,
+//     rounded to bf16, in shared memory as the B operand of the next
 //     chunk.  The critical path per chunk is two tensor-core round trips
 //     (V', then D4) and two short epilogues; -W is formed before S is needed,
 //     and the output rows (P V' + Q S) are finished by warps 10-11 while
@@ -28,11 +29,9 @@
 //   G  = [K; Q] K^T                                     tcgen05 M=128 N=64 K=128
 //   A  = -strictLower(diag(beta rk) (K K^T) diag(rk) * Gamma)          CUDA cores
 //   P  = diag(rq) (Q K^T) diag(rk) * Gamma  (lower incl. diagonal)      CUDA cores
-//   T  = (I - A)^-1 = R + N^2 R,  R = T_D + N T_D,  N = T_D A_off       3 tcgen05 rounds
-//        (T_D: inverse of A's 16x16 diagonal blocks, one column per lane by
-//        forward substitution; A_off: the strictly block-lower part of A;
-//        N^4 = 0.  The 16-row block scheme is the PyPTO README's inverse_pto
-//        submodule.)
+//   T  = (I - A)^-1 over 32 x 32 blocks, fp32 in shared memory:     CUDA cores
+//        T11, T22 by forward substitution on T = I + A T (one column per lane),
+//        T21 = T22 (A21 T11) (two 32 x 32 products over 256 threads)
 //   serial:  -W = (-T diag(beta exp(gcum) rk)) K                        one round
 //            V' = T diag(beta) V + (-W) S   (one accumulator)           one round
 //            [KS; QS] = [K; Q] S                                  same round, own use
@@ -79,17 +78,15 @@ constexpr int PS_WLO = 0, PS_WHI = 1 * kTile, PS_P = 2 * kTile, PS_TU = 3 * kTil
 constexpr int kProd = 4 * kTile;
 constexpr int OFF_RAW = 0;
 constexpr int OFF_PROD = NR * kRaw;
-constexpr int OFF_X0 = OFF_PROD + NP * kProd;  // intra scratch: A_off, N, N^2
-constexpr int OFF_X1 = OFF_X0 + kTile;         // intra scratch: T_D, R
-constexpr int OFF_S = OFF_X1 + kTile;          // serial: S operand, 128 rows (d) x 64 cols
+// intra scratch M: fp32 64 x 64 with rows padded to MS_LD floats, holding A^T,
+// then the blocks of T = (I - A)^-1
+constexpr int MS_LD = 68;
+constexpr int OFF_MS = OFF_PROD + NP * kProd;
+constexpr int OFF_S = OFF_MS + 64 * MS_LD * 4;  // serial: S operand, 128 rows (d) x 64 cols
 constexpr int OFF_SCI = OFF_S + 2 * kTile;     // intra scalars
 constexpr int SI_RK = 0, SI_RQ = 64, SI_BETA = 128, SI_GC = 192, SI_BW = 256, SI_NP = 320, SI_WK = 576,
               SI_SQ = 640, SI_GAM = 704, SI_CF = 708, SI_N = 772;
-// diagonal 16 x 16 blocks of A, then of T_D, as fp32 (4 blocks, padded so the
-// two blocks a warp handles sit in different banks)
-constexpr int LS_BLK = 16 * 16 + 16;
-constexpr int OFF_LS = OFF_SCI + SI_N * 4;
-constexpr int OFF_SCP = OFF_LS + 4 * LS_BLK * 4;  // per-product-slot scalars for the serial side
+constexpr int OFF_SCP = OFF_SCI + SI_N * 4;    // per-product-slot scalars for the serial side
 constexpr int SP_WK = 0, SP_SQ = 64, SP_GAMMA = 128, SP_N = 132;
 // bytes one CTA sends to the other per chunk it builds: -T diag(bw), P, T diag(beta), wk, sq, gamma
 constexpr uint32_t kPushBytes = 3 * 8192 + (2 * 64 + 1) * 4;
@@ -106,8 +103,8 @@ static_assert(OFF_BAR % 8 == 0, "mbarrier alignment");
 static_assert(SMEM_BYTES <= 232448, "shared memory");
 
 // ---- TMEM columns (128 lanes x 512 fp32 columns)
-constexpr uint32_t TM_G = 0;     // intra: G; then N; then N^2 R
-constexpr uint32_t TM_N2 = 64;   // intra: [N^2 | N T_D] (128 cols)
+constexpr uint32_t TM_G = 0;     // intra: G
+constexpr uint32_t TM_S = 64;    // serial: the fp32 state slice S (row d in lane d, 64 cols)
 constexpr uint32_t TM_QS = 192;  // serial: [K S ; Q S], two column blocks used alternately (128 cols)
 constexpr uint32_t TM_W = 320;   // serial: -W (128 cols: the U and D4 blocks, both free at that point)
 constexpr uint32_t TM_U = 320;   // serial: U - W S (rows 0..63)
@@ -237,9 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = row & 63;
     const int c0 = 32 * hf;
     const bool krow = q < 2;
-    // the 16x16 diagonal block of key row r lies in this thread's half
-    const bool diag_here = krow && ((r >> 5) == hf);
-    const int li = lane & 15;
+    float* ms = reinterpret_cast<float*>(sm + OFF_MS);
     uint32_t ph_mma = 0;
     bool ok = true;
     // One thread polls the mbarrier; the others park at the named barrier.
@@ -248,25 +243,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = !named_bar_any(1, 256, *abort_flag != 0);
       ptx::tc_fence_after();
     };
-    auto wait_mma = [&]() {
-      wait_bar(bars + BAR_MMAI, ph_mma);
-      ph_mma ^= 1u;
-    };
-    auto publish = [&]() {
-      ptx::fence_proxy_async_smem();
-      ptx::tc_fence_before();
-      named_bar_n(1, 256);
-    };
-    // this thread's 32 columns of T_D (block-diagonal inverse) for key row r
-    auto td_half = [&](const float* t16, float* out32) {
-#pragma unroll
-      for (int cc = 0; cc < 32; ++cc) {
-        const int cj = cc & 15;
-        const bool same_block = (cc >> 4) == (lane >> 4);
-        out32[cc] = (diag_here && same_block) ? (cj < li ? t16[cj] : (cj == li ? 1.f : 0.f)) : 0.f;
-      }
-    };
-
     float g_next = 0.f, b_next = 0.f;
     {
       const int64_t t0g = seq_start + (int64_t)crank * C + t;
@@ -352,11 +328,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         si[SI_SQ + t] = eg * si[SI_RQ + t];
         if (t == 0) si[SI_GAM] = fast_exp(gl);
       }
-      wait_mma();  // G ready (the named barrier inside also publishes the scalars)
+      wait_bar(bars + BAR_MMAI, ph_mma);  // G ready (the barrier also publishes the scalars)
+      ph_mma ^= 1u;
       if (!ok) break;
-      // A rows (key rows) with the diagonal-block inverse; P rows (query rows)
-      float keep[32];  // key rows: R = T_D + N T_D (this half); query rows: this half of P
-      float t16[16];   // diagonal-block threads: strictly lower part of this row's T_D block
+      // A rows (key rows) go to the fp32 scratch M for the inverse; P rows
+      // (query rows) wait in registers, packed to bf16, until the slot is free
+      uint4 pk0[4];
       {
         // G row r, columns [c0, c0 + 32), scaled to A (key rows) or P (query rows):
         //   A[r][i] = -beta_r rk_r rk_i exp(gcum_r - gcum_i) (K K^T)[r][i],  i < r
@@ -367,6 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float av[32];
         ptx::tmem_ld32(tl + TM_G + c0, av);
         ptx::tmem_ld_wait();
+        ptx::tc_fence_before();  // G is consumed: the next chunk's G may overwrite it after any barrier
         const float f = krow ? -si[SI_BETA + r] * si[SI_RK + r] : si[SI_RQ + r];
         const int rblk = r >> 5;  // == q & 1: warp-uniform
         if (rblk > hf) {
@@ -399,99 +377,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int cc = 0; cc < 32; ++cc) av[cc] = 0.f;
         }
         if (krow) {
-          if (diag_here) {
-            // T_D = (I - A_D)^-1 for this warp's two 16 x 16 diagonal blocks
-            // (lanes 0-15: block 2 rblk, lanes 16-31: block 2 rblk + 1).  Lane li
-            // first publishes row li of A_D column-major, then solves column li of
-            // T_D = I + A_D T_D top to bottom, then reads back row li of T_D.
-            float* ls = reinterpret_cast<float*>(sm + OFF_LS) + (2 * rblk + (lane >> 4)) * LS_BLK;
+          if (rblk >= hf) {  // the 32 x 32 block above the diagonal is zero and never read
+            float* mc = ms + c0 * MS_LD + r;  // M[i][r] = A[r][i]: column i of A is row i of M
 #pragma unroll
-            for (int k = 0; k < 16; ++k) ls[k * 16 + li] = lane < 16 ? av[k] : av[16 + k];  // A_D[li][k] (0 for k >= li)
-            __syncwarp();
-            float x[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) x[i] = (i == li) ? 1.f : 0.f;
-#pragma unroll
-            for (int k = 0; k < 15; ++k) {
-              float colk[16];
-              const float4* c4 = reinterpret_cast<const float4*>(ls + k * 16);
-#pragma unroll
-              for (int v = 0; v < 4; ++v) {
-                const float4 y = c4[v];
-                colk[4 * v] = y.x; colk[4 * v + 1] = y.y; colk[4 * v + 2] = y.z; colk[4 * v + 3] = y.w;
-              }
-#pragma unroll
-              for (int i = k + 1; i < 16; ++i) x[i] = fmaf(colk[i], x[k], x[i]);
-            }
-            __syncwarp();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) ls[i * 16 + li] = x[i];  // T_D[i][li], now row-major
-            __syncwarp();
-            const float4* r4 = reinterpret_cast<const float4*>(ls + li * 16);
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              const float4 y = r4[v];
-              t16[4 * v] = y.x; t16[4 * v + 1] = y.y; t16[4 * v + 2] = y.z; t16[4 * v + 3] = y.w;
-            }
+            for (int cc = 0; cc < 32; ++cc) mc[cc * MS_LD] = av[cc];
           }
-          td_half(t16, keep);
-          ptx::st_half_bf16(sm + OFF_X1, r, hf, keep);  // T_D
-          const int bcol = 16 * (r >> 4);
-#pragma unroll
-          for (int cc = 0; cc < 32; ++cc) av[cc] = (c0 + cc < bcol) ? av[cc] : 0.f;
-          ptx::st_half_bf16(sm + OFF_X0, r, hf, av);  // A_off
         } else {
-#pragma unroll
-          for (int cc = 0; cc < 32; ++cc) keep[cc] = av[cc];  // P, stored once the slot is free
+          ptx::pack_half_bf16(av, pk0);  // P
         }
       }
-      publish();
-      // N = T_D A_off   (A = [T_D; junk]: rows land in lanes 0..63)
-      if (t == 0) {
-        ptx::tc_fence_after();
-        mma_k64(tmem + TM_G, sb + OFF_X1, sb + OFF_X0, 8192, ID_KMN64, 0);
-        ptx::mma_commit(bars + BAR_MMAI);
-      }
-      wait_mma();
-      if (!ok) break;
-      if (krow) {
-        float x[32];
-        ptx::tmem_ld32(tl + TM_G + c0, x);
-        ptx::tmem_ld_wait();
-        ptx::st_half_bf16(sm + OFF_X0, r, hf, x);  // N (A_off has been consumed)
-      }
-      publish();
-      // [N^2 | N T_D] = N [N | T_D]
-      if (t == 0) {
-        ptx::tc_fence_after();
-        mma_k64(tmem + TM_N2, sb + OFF_X0, sb + OFF_X0, OFF_X1 - OFF_X0, ID_KMN128, 0);
-        ptx::mma_commit(bars + BAR_MMAI);
-      }
-      wait_mma();
-      if (!ok) break;
-      if (krow) {
-        float x[32];
-        ptx::tmem_ld32(tl + TM_N2 + c0, x);
-        ptx::tmem_ld_wait();
-        ptx::st_half_bf16(sm + OFF_X0, r, hf, x);  // N^2
-        ptx::tmem_ld32(tl + TM_N2 + 64 + c0, x);
-        ptx::tmem_ld_wait();
-        td_half(t16, keep);
-#pragma unroll
-        for (int cc = 0; cc < 32; ++cc) keep[cc] += x[cc];  // R = T_D + N T_D
-        ptx::st_half_bf16(sm + OFF_X1, r, hf, keep);  // R (T_D has been consumed)
-      }
-      publish();
-      // N^2 R
-      if (t == 0) {
-        ptx::tc_fence_after();
-        mma_k64(tmem + TM_G, sb + OFF_X0, sb + OFF_X1, 8192, ID_KMN64, 0);
-        ptx::mma_commit(bars + BAR_MMAI);
-      }
       // the product slot (both copies) must have been released by both CTAs'
-      // serial warps (chunk c - 2) before the products are stored
+      // serial warps (chunk c - 2) before this chunk's products are stored
       if (t == 0) {
-        if (!ptx::mbar_wait_bounded(bars + BAR_MMAI, ph_mma, kWaitNs)) *abort_flag = 1;
         if (c >= NP) {
           const uint32_t par = (uint32_t)((c / NP - 1) & 1);
           if (!ptx::mbar_wait_bounded(bars + BAR_PRODE + psl, par, kWaitNs)) *abort_flag = 1;
@@ -499,49 +396,119 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (*abort_flag == 0) ptx::mbar_arrive_expect_tx_remote(rbar, kPushBytes);  // arm the other CTA's copy
       }
-      ph_mma ^= 1u;
-      ok = !named_bar_any(1, 256, *abort_flag != 0);
-      ptx::tc_fence_after();
+      ok = !named_bar_any(1, 256, *abort_flag != 0);  // also: A^T is in M
       if (!ok) break;
+      // T = (I - A)^-1 over 32 x 32 blocks, in fp32 on the CUDA cores
+      // (A is strictly lower triangular, so T is unit lower triangular):
+      //   T11 = (I - A11)^-1, T22 = (I - A22)^-1: one column per lane (warps 0, 1),
+      //     from T = I + A T top to bottom; each replaces A^T in its block of M
+      //   Y = A21 T11 into M's block (1,0), then T21 = T22 Y over A21^T in block (0,1)
+      if (warp < 2) {
+        const int w = warp;
+        float* mb = ms + 32 * w * MS_LD + 32 * w;  // block (w, w); row k = column k of A_ww
+        float x[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[i] = (i == lane) ? 1.f : 0.f;
+        // column k of A_ww (rows > k) is loaded one step ahead of its use
+        float4 cur[8], nxt[8];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) cur[v] = *reinterpret_cast<const float4*>(mb + 4 * v);
+#pragma unroll
+        for (int k = 0; k < 31; ++k) {
+          if (k + 1 < 31) {
+#pragma unroll
+            for (int v = (k + 2) >> 2; v < 8; ++v)
+              nxt[v] = *reinterpret_cast<const float4*>(mb + (k + 1) * MS_LD + 4 * v);
+          }
+#pragma unroll
+          for (int i = k + 1; i < 32; ++i) {
+            const float4 y = cur[i >> 2];
+            const float aik = (i & 3) == 0 ? y.x : (i & 3) == 1 ? y.y : (i & 3) == 2 ? y.z : y.w;
+            x[i] = fmaf(aik, x[k], x[i]);
+          }
+#pragma unroll
+          for (int v = 0; v < 8; ++v) cur[v] = nxt[v];
+        }
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) mb[i * MS_LD + lane] = x[i];  // T_ww, row-major
+      }
+      named_bar_n(1, 256);
+      {
+        // Y[i][j] = sum_k A21[i][k] T11[k][j] = sum_k M[k][32 + i] M[k][j]
+        const int i = t >> 3, j4 = 4 * (t & 7);
+        float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          const float a21 = ms[k * MS_LD + 32 + i];
+          const float4 t11 = *reinterpret_cast<const float4*>(ms + k * MS_LD + j4);
+          y0 = fmaf(a21, t11.x, y0);
+          y1 = fmaf(a21, t11.y, y1);
+          y2 = fmaf(a21, t11.z, y2);
+          y3 = fmaf(a21, t11.w, y3);
+        }
+        *reinterpret_cast<float4*>(ms + (32 + i) * MS_LD + j4) = make_float4(y0, y1, y2, y3);
+      }
+      named_bar_n(1, 256);
+      {
+        // T21[i][j] = sum_k T22[i][k] Y[k][j] = sum_k M[32 + i][32 + k] M[32 + k][j]
+        const int i = t >> 3, j4 = 4 * (t & 7);
+        float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          const float t22 = ms[(32 + i) * MS_LD + 32 + k];
+          const float4 yk = *reinterpret_cast<const float4*>(ms + (32 + k) * MS_LD + j4);
+          y0 = fmaf(t22, yk.x, y0);
+          y1 = fmaf(t22, yk.y, y1);
+          y2 = fmaf(t22, yk.z, y2);
+          y3 = fmaf(t22, yk.w, y3);
+        }
+        *reinterpret_cast<float4*>(ms + i * MS_LD + 32 + j4) = make_float4(y0, y1, y2, y3);
+      }
+      named_bar_n(1, 256);  // T21 is in M
       // products: stored locally first (and made visible to this CTA's tensor
       // cores), then sent to the other CTA with st.async
-      uint4 pk0[4], pk1[4];
       if (t < 64) {
         spp[SP_WK + t] = si[SI_WK + t];
         spp[SP_SQ + t] = si[SI_SQ + t];
         if (t == 0) spp[SP_GAMMA] = si[SI_GAM];
       }
       if (!krow) {
-        ptx::pack_half_bf16(keep, pk0);  // P
-        ptx::st_half_packed(ps + PS_P, r, hf, pk0);
-      } else {
-        float x[32];
-        ptx::tmem_ld32(tl + TM_G + c0, x);
-        ptx::tmem_ld_wait();
-#pragma unroll
-        for (int cc = 0; cc < 32; ++cc) x[cc] += keep[cc];  // T = R + N^2 R
-#pragma unroll
-        for (int cc = 0; cc < 32; ++cc) keep[cc] = -x[cc] * si[SI_BW + c0 + cc];
-        ptx::pack_half_bf16(keep, pk0);  // -T diag(beta exp(gcum) rk), for W
-        ptx::st_half_packed(ps + PS_WHI, r, hf, pk0);
-#pragma unroll
-        for (int cc = 0; cc < 32; ++cc) keep[cc] = x[cc] * si[SI_BETA + c0 + cc];
-        ptx::pack_half_bf16(keep, pk1);  // T diag(beta), for U
-        ptx::st_half_packed(ps + PS_TU, r, hf, pk1);
-      }
-      ptx::fence_proxy_async_smem();
-      if (t < 64) {
-        ptx::st_async_b32(rspp + 4 * (SP_WK + t), __float_as_uint(si[SI_WK + t]), rbar);
-        ptx::st_async_b32(rspp + 4 * (SP_SQ + t), __float_as_uint(si[SI_SQ + t]), rbar);
-        if (t == 0) ptx::st_async_b32(rspp + 4 * SP_GAMMA, __float_as_uint(si[SI_GAM]), rbar);
-      }
-      if (!krow) {
+        ptx::st_half_packed(ps + PS_P, r, hf, pk0);  // P
+        ptx::fence_proxy_async_smem();
         ptx::st_half_packed_remote(rpa + PS_P, rbar, r, hf, pk0);
       } else {
+        uint4 pk1[4];
+        float x[32];  // row r of T, columns [c0, c0 + 32)
+        if (r < 32 && hf == 1) {
+#pragma unroll
+          for (int cc = 0; cc < 32; ++cc) x[cc] = 0.f;
+        } else {
+          const float* tr = ms + (r < 32 ? r * MS_LD : (hf == 0 ? (r - 32) * MS_LD + 32 : r * MS_LD + 32));
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            const float4 y = *reinterpret_cast<const float4*>(tr + 4 * v);
+            x[4 * v] = y.x; x[4 * v + 1] = y.y; x[4 * v + 2] = y.z; x[4 * v + 3] = y.w;
+          }
+        }
+        float y[32];
+#pragma unroll
+        for (int cc = 0; cc < 32; ++cc) y[cc] = -x[cc] * si[SI_BW + c0 + cc];
+        ptx::pack_half_bf16(y, pk0);  // -T diag(beta exp(gcum) rk), for W
+        ptx::st_half_packed(ps + PS_WHI, r, hf, pk0);
+#pragma unroll
+        for (int cc = 0; cc < 32; ++cc) y[cc] = x[cc] * si[SI_BETA + c0 + cc];
+        ptx::pack_half_bf16(y, pk1);  // T diag(beta), for U
+        ptx::st_half_packed(ps + PS_TU, r, hf, pk1);
+        ptx::fence_proxy_async_smem();
+        if (t < 64) {
+          ptx::st_async_b32(rspp + 4 * (SP_WK + t), __float_as_uint(si[SI_WK + t]), rbar);
+          ptx::st_async_b32(rspp + 4 * (SP_SQ + t), __float_as_uint(si[SI_SQ + t]), rbar);
+          if (t == 0) ptx::st_async_b32(rspp + 4 * SP_GAMMA, __float_as_uint(si[SI_GAM]), rbar);
+        }
         ptx::st_half_packed_remote(rpa + PS_WHI, rbar, r, hf, pk0);
         ptx::st_half_packed_remote(rpa + PS_TU, rbar, r, hf, pk1);
       }
-      ptx::tc_fence_before();
       named_bar_n(1, 256);
       if (t == 0) ptx::mbar_arrive(bars + BAR_PRODF + psl);  // the other CTA's copy completes by transactions
     }
@@ -551,20 +518,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     // serial warps (8-11)
     // =====================================================================
     const int t = tid - 256;  // 0..127: row d of the state
-    float S[64];
+    // S lives in TMEM (fp32) and, rounded to bf16, in shared memory
     const size_t st_off = ((size_t)n * nv + h) * (size_t)DK * dv + (size_t)t * dv + slice * DVS;
-    if (a.s0) {
-      const float4* src = reinterpret_cast<const float4*>(a.s0 + st_off);
 #pragma unroll
-      for (int cc = 0; cc < 16; ++cc) {
-        const float4 x = src[cc];
-        S[4 * cc] = x.x; S[4 * cc + 1] = x.y; S[4 * cc + 2] = x.z; S[4 * cc + 3] = x.w;
+    for (int hh = 0; hh < 2; ++hh) {
+      float x[32];
+      if (a.s0) {
+        const float4* src = reinterpret_cast<const float4*>(a.s0 + st_off + 32 * hh);
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          const float4 y = src[cc];
+          x[4 * cc] = y.x; x[4 * cc + 1] = y.y; x[4 * cc + 2] = y.z; x[4 * cc + 3] = y.w;
+        }
+      } else {
+#pragma unroll
+        for (int cc = 0; cc < 32; ++cc) x[cc] = 0.f;
       }
-    } else {
-#pragma unroll
-      for (int cc = 0; cc < 64; ++cc) S[cc] = 0.f;
+      ptx::tmem_st32(tl + TM_S + 32 * hh, x);
+      ptx::st_half_bf16(sm + OFF_S, t, hh, x);
     }
-    ptx::st_row_bf16(sm + OFF_S, t, S);
+    ptx::tmem_st_wait();
     ptx::fence_proxy_async_smem();
     named_bar_n(2, 128);
 
@@ -685,13 +658,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float decay = spp[SP_GAMMA];
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
-          float x[32];
+          float x[32], sv[32];
           ptx::tmem_ld32(tl + TM_D4 + 32 * hh, x);
+          ptx::tmem_ld32(tl + TM_S + 32 * hh, sv);
           ptx::tmem_ld_wait();
 #pragma unroll
-          for (int cc = 0; cc < 32; ++cc) S[32 * hh + cc] = fmaf(decay, S[32 * hh + cc], x[cc]);
+          for (int cc = 0; cc < 32; ++cc) sv[cc] = fmaf(decay, sv[cc], x[cc]);
+          ptx::tmem_st32(tl + TM_S + 32 * hh, sv);
+          ptx::st_half_bf16(sm + OFF_S, t, hh, sv);
         }
-        ptx::st_row_bf16(sm + OFF_S, t, S);
+        ptx::tmem_st_wait();
       }
       ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
@@ -755,9 +731,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::mbar_wait_bounded(bars + BAR_RAWF + cn % NR, (uint32_t)((cn / NR) & 1), kWaitNs);
     }
     if (ok && a.s_final) {
-      float4* dst = reinterpret_cast<float4*>(a.s_final + st_off);
 #pragma unroll
-      for (int cc = 0; cc < 16; ++cc) dst[cc] = make_float4(S[4 * cc], S[4 * cc + 1], S[4 * cc + 2], S[4 * cc + 3]);
+      for (int hh = 0; hh < 2; ++hh) {
+        float x[32];
+        ptx::tmem_ld32(tl + TM_S + 32 * hh, x);
+        ptx::tmem_ld_wait();
+        float4* dst = reinterpret_cast<float4*>(a.s_final + st_off + 32 * hh);
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) dst[cc] = make_float4(x[4 * cc], x[4 * cc + 1], x[4 * cc + 2], x[4 * cc + 3]);
+      }
     }
     if (!ok && t == 0) atomicOr(&g_status, 1u);
   }
