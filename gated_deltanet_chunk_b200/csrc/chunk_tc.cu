@@ -434,36 +434,53 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 32; ++i) mb[i * MS_LD + lane] = x[i];  // T_ww, row-major
       }
       named_bar_n(1, 256);
-      {
+      // Y = A21 T11 and T21 = T22 Y on warps 0-3 (one per scheduler): each of
+      // 128 threads owns a 2 x 4 output tile
+      const int i2 = 2 * (t >> 3), j4 = 4 * (t & 7);
+      if (warp < 4) {
         // Y[i][j] = sum_k A21[i][k] T11[k][j] = sum_k M[k][32 + i] M[k][j]
-        const int i = t >> 3, j4 = 4 * (t & 7);
-        float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
+        float y[2][4] = {};
 #pragma unroll
         for (int k = 0; k < 32; ++k) {
-          const float a21 = ms[k * MS_LD + 32 + i];
-          const float4 t11 = *reinterpret_cast<const float4*>(ms + k * MS_LD + j4);
-          y0 = fmaf(a21, t11.x, y0);
-          y1 = fmaf(a21, t11.y, y1);
-          y2 = fmaf(a21, t11.z, y2);
-          y3 = fmaf(a21, t11.w, y3);
+          const float2 a = *reinterpret_cast<const float2*>(ms + k * MS_LD + 32 + i2);
+          const float4 b = *reinterpret_cast<const float4*>(ms + k * MS_LD + j4);
+          const float av2[2] = {a.x, a.y}, bv4[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+          for (int r2 = 0; r2 < 2; ++r2)
+#pragma unroll
+            for (int c2 = 0; c2 < 4; ++c2) y[r2][c2] = fmaf(av2[r2], bv4[c2], y[r2][c2]);
         }
-        *reinterpret_cast<float4*>(ms + (32 + i) * MS_LD + j4) = make_float4(y0, y1, y2, y3);
+#pragma unroll
+        for (int r2 = 0; r2 < 2; ++r2)
+          *reinterpret_cast<float4*>(ms + (32 + i2 + r2) * MS_LD + j4) = make_float4(y[r2][0], y[r2][1], y[r2][2], y[r2][3]);
       }
       named_bar_n(1, 256);
-      {
+      if (warp < 4) {
         // T21[i][j] = sum_k T22[i][k] Y[k][j] = sum_k M[32 + i][32 + k] M[32 + k][j]
-        const int i = t >> 3, j4 = 4 * (t & 7);
-        float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
+        float y[2][4] = {};
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          const float t22 = ms[(32 + i) * MS_LD + 32 + k];
-          const float4 yk = *reinterpret_cast<const float4*>(ms + (32 + k) * MS_LD + j4);
-          y0 = fmaf(t22, yk.x, y0);
-          y1 = fmaf(t22, yk.y, y1);
-          y2 = fmaf(t22, yk.z, y2);
-          y3 = fmaf(t22, yk.w, y3);
+        for (int k4 = 0; k4 < 32; k4 += 4) {
+          float a[2][4], b[4][4];
+#pragma unroll
+          for (int r2 = 0; r2 < 2; ++r2) {
+            const float4 v = *reinterpret_cast<const float4*>(ms + (32 + i2 + r2) * MS_LD + 32 + k4);
+            a[r2][0] = v.x; a[r2][1] = v.y; a[r2][2] = v.z; a[r2][3] = v.w;
+          }
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const float4 v = *reinterpret_cast<const float4*>(ms + (32 + k4 + kk) * MS_LD + j4);
+            b[kk][0] = v.x; b[kk][1] = v.y; b[kk][2] = v.z; b[kk][3] = v.w;
+          }
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+            for (int r2 = 0; r2 < 2; ++r2)
+#pragma unroll
+              for (int c2 = 0; c2 < 4; ++c2) y[r2][c2] = fmaf(a[r2][kk], b[kk][c2], y[r2][c2]);
         }
-        *reinterpret_cast<float4*>(ms + i * MS_LD + 32 + j4) = make_float4(y0, y1, y2, y3);
+#pragma unroll
+        for (int r2 = 0; r2 < 2; ++r2)
+          *reinterpret_cast<float4*>(ms + (i2 + r2) * MS_LD + 32 + j4) = make_float4(y[r2][0], y[r2][1], y[r2][2], y[r2][3]);
       }
       named_bar_n(1, 256);  // T21 is in M
       // products: stored locally first (and made visible to this CTA's tensor
