@@ -149,19 +149,6 @@ __device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t cluster_ba
                "r"(bytes)
                : "memory");
 }
-// Bulk copy of `bytes` (a multiple of 16; both addresses 16-byte aligned) from
-// this CTA's shared memory to another CTA's (`dst` is a shared::cluster
-// address), completing `bytes` of transaction count on that CTA's mbarrier.
-// No multicast.
-__device__ __forceinline__ void bulk_copy_to_cta(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t cluster_bar) {
-  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                   dst),
-               "r"(src), "r"(bytes), "r"(cluster_bar)
-               : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// waits until the source reads of every committed bulk copy of this thread are done
-__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
