@@ -59,6 +59,13 @@ def lib() -> ctypes.CDLL:
         L.gdn_recurrent_step.argtypes = [vp, vp, vp, fp, fp, fp, vp, ctypes.c_int32,
                                          ctypes.POINTER(GdnParams), vp]
         L.gdn_recurrent_step.restype = ctypes.c_int
+        L.gdn_chunk_fwd_gated.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, ip, ctypes.c_int32,
+                                          ctypes.c_int64, ctypes.c_int32, vp, fp,
+                                          ctypes.POINTER(GdnParams), vp]
+        L.gdn_chunk_fwd_gated.restype = ctypes.c_int
+        L.gdn_recurrent_step_gated.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, vp, ctypes.c_int32,
+                                               ctypes.POINTER(GdnParams), vp]
+        L.gdn_recurrent_step_gated.restype = ctypes.c_int
         L.gdn_device_status.argtypes = [vp]
         L.gdn_device_status.restype = ctypes.c_int
         L.gdn_status_string.argtypes = [ctypes.c_int]
@@ -84,6 +91,25 @@ def make_params(nqk, nv, dk, dv, io_bf16, qk_l2norm=True, scale=0.0, kernel="aut
                      1 if qk_l2norm else 0, float(scale), KERNELS[kernel])
 
 
+def _chunk_call(name, gate, q, k, v, initial_state, cu_seqlens, chunk_size, out, final_state,
+                output_final_state, num_seqs, qk_l2norm, scale, kernel, stream, check):
+    import torch
+    T, nqk, dk = q.shape
+    nv, dv = v.shape[1], v.shape[2]
+    n = (cu_seqlens.numel() - 1) if cu_seqlens is not None else (num_seqs or 1)
+    if out is None:
+        out = torch.empty((T, nv, dv), dtype=v.dtype, device=v.device)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((n, nv, dk, dv), dtype=torch.float32, device=v.device)
+    p = make_params(nqk, nv, dk, dv, q.dtype == torch.bfloat16, qk_l2norm, scale, kernel)
+    rc = getattr(lib(), name)(_ptr(q), _ptr(k), _ptr(v), *[_ptr(x) for x in gate], _ptr(initial_state),
+                              _ptr(cu_seqlens), int(n), int(T), int(chunk_size), _ptr(out),
+                              _ptr(final_state), ctypes.byref(p), _stream(stream))
+    if check and rc != GDN_OK:
+        raise GdnError(rc, name)
+    return out, final_state
+
+
 def chunk_fwd(q, k, v, g, beta, initial_state=None, cu_seqlens=None, chunk_size=64,
               out=None, final_state=None, output_final_state=True, num_seqs=None,
               qk_l2norm=True, scale=0.0, kernel="auto", stream=None, check=True):
@@ -94,21 +120,37 @@ def chunk_fwd(q, k, v, g, beta, initial_state=None, cu_seqlens=None, chunk_size=
     cu_seqlens [N+1] int32 or None (then ``num_seqs`` equal sequences, default 1).
     Returns ``(out, final_state)``; final_state is None when not requested.
     """
+    return _chunk_call("gdn_chunk_fwd", (g, beta), q, k, v, initial_state, cu_seqlens, chunk_size,
+                       out, final_state, output_final_state, num_seqs, qk_l2norm, scale, kernel,
+                       stream, check)
+
+
+def chunk_fwd_gated(q, k, v, a, b, A_log, dt_bias, initial_state=None, cu_seqlens=None,
+                    chunk_size=64, out=None, final_state=None, output_final_state=True,
+                    num_seqs=None, qk_l2norm=True, scale=0.0, kernel="auto", stream=None,
+                    check=True):
+    """``chunk_fwd`` with the gate formed in-kernel (``gdn_chunk_fwd_gated``).
+
+    a, b [T, Nv] fp32 raw projections; A_log, dt_bias [Nv] fp32:
+    beta = sigmoid(b), g = -exp(A_log) * softplus(a + dt_bias).
+    """
+    return _chunk_call("gdn_chunk_fwd_gated", (a, b, A_log, dt_bias), q, k, v, initial_state,
+                       cu_seqlens, chunk_size, out, final_state, output_final_state, num_seqs,
+                       qk_l2norm, scale, kernel, stream, check)
+
+
+def _step_call(name, gate, q, k, v, state, out, qk_l2norm, scale, stream, check):
     import torch
-    T, nqk, dk = q.shape
+    N, nqk, dk = q.shape
     nv, dv = v.shape[1], v.shape[2]
-    n = (cu_seqlens.numel() - 1) if cu_seqlens is not None else (num_seqs or 1)
     if out is None:
-        out = torch.empty((T, nv, dv), dtype=v.dtype, device=v.device)
-    if final_state is None and output_final_state:
-        final_state = torch.empty((n, nv, dk, dv), dtype=torch.float32, device=v.device)
-    p = make_params(nqk, nv, dk, dv, q.dtype == torch.bfloat16, qk_l2norm, scale, kernel)
-    rc = lib().gdn_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state),
-                             _ptr(cu_seqlens), int(n), int(T), int(chunk_size), _ptr(out),
-                             _ptr(final_state), ctypes.byref(p), _stream(stream))
+        out = torch.empty((N, nv, dv), dtype=v.dtype, device=v.device)
+    p = make_params(nqk, nv, dk, dv, q.dtype == torch.bfloat16, qk_l2norm, scale)
+    rc = getattr(lib(), name)(_ptr(q), _ptr(k), _ptr(v), *[_ptr(x) for x in gate], _ptr(state),
+                              _ptr(out), int(N), ctypes.byref(p), _stream(stream))
     if check and rc != GDN_OK:
-        raise GdnError(rc, "gdn_chunk_fwd")
-    return out, final_state
+        raise GdnError(rc, name)
+    return out
 
 
 def recurrent_step(q, k, v, g, beta, state, out=None, qk_l2norm=True, scale=0.0, stream=None,
@@ -118,17 +160,18 @@ def recurrent_step(q, k, v, g, beta, state, out=None, qk_l2norm=True, scale=0.0,
     q, k [N, Nqk, Dk], v [N, Nv, Dv], g, beta [N, Nv], state [N, Nv, Dk, Dv] fp32.
     Returns out [N, Nv, Dv].
     """
-    import torch
-    N, nqk, dk = q.shape
-    nv, dv = v.shape[1], v.shape[2]
-    if out is None:
-        out = torch.empty((N, nv, dv), dtype=v.dtype, device=v.device)
-    p = make_params(nqk, nv, dk, dv, q.dtype == torch.bfloat16, qk_l2norm, scale)
-    rc = lib().gdn_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state),
-                                  _ptr(out), int(N), ctypes.byref(p), _stream(stream))
-    if check and rc != GDN_OK:
-        raise GdnError(rc, "gdn_recurrent_step")
-    return out
+    return _step_call("gdn_recurrent_step", (g, beta), q, k, v, state, out, qk_l2norm, scale,
+                      stream, check)
+
+
+def recurrent_step_gated(q, k, v, a, b, A_log, dt_bias, state, out=None, qk_l2norm=True,
+                         scale=0.0, stream=None, check=True):
+    """``recurrent_step`` with the gate formed in-kernel (``gdn_recurrent_step_gated``).
+
+    a, b [N, Nv] fp32 raw projections; A_log, dt_bias [Nv] fp32.
+    """
+    return _step_call("gdn_recurrent_step_gated", (a, b, A_log, dt_bias), q, k, v, state, out,
+                      qk_l2norm, scale, stream, check)
 
 
 def device_status(stream=None) -> int:

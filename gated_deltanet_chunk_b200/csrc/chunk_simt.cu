@@ -170,8 +170,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_simt_kernel(ChunkArgs a
     if (tid < C) {
       const int64_t t = c0 + tid;
       const bool valid = t < seq_end;
-      gc[tid] = valid ? a.g[(size_t)t * nv + h] : 0.f;
-      bt[tid] = valid ? a.beta[(size_t)t * nv + h] : 0.f;
+      float gv = 0.f, bv = 0.f;
+      if (valid) load_gate(a, (size_t)t * nv + h, h, gv, bv);
+      gc[tid] = gv;
+      bt[tid] = bv;
     }
     __syncthreads();
     // ---- in-chunk inclusive cumsum of g (one warp) ----

@@ -247,8 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     {
       const int64_t t0g = seq_start + (int64_t)crank * C + t;
       if (t < 64 && t0g < seq_end) {
-        g_next = a.g[(size_t)t0g * nv + h];
-        b_next = a.beta[(size_t)t0g * nv + h];
+        load_gate(a, (size_t)t0g * nv + h, h, g_next, b_next);
       }
     }
 
@@ -279,8 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         g_next = 0.f;
         b_next = 0.f;
         if (tn < seq_end) {
-          g_next = a.g[(size_t)tn * nv + h];
-          b_next = a.beta[(size_t)tn * nv + h];
+          load_gate(a, (size_t)tn * nv + h, h, g_next, b_next);
         }
       }
       wait_bar(bars + BAR_RAWF + rsl, (uint32_t)((c / NR) & 1));

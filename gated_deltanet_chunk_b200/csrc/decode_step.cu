@@ -45,8 +45,9 @@ __global__ void __launch_bounds__(kThreads, 2) recurrent_step_kernel(StepArgs a)
 #pragma unroll
   for (int i = 0; i < RPT; ++i) s[i] = __ldcs(st + (size_t)(i * RG + rg) * CG + cg);
 
-  const float alpha = expf(a.g[(size_t)n * a.nv + h]);
-  const float bta = a.beta[(size_t)n * a.nv + h];
+  float gv, bta;
+  load_gate(a, (size_t)n * a.nv + h, h, gv, bta);
+  const float alpha = expf(gv);
 
   // q_hat, k_hat (warp 0: q, warp 1: k)
   if (warp < 2) {

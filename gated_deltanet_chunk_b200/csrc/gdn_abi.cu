@@ -15,6 +15,7 @@ namespace {
 constexpr int kMaxDevices = 64;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 struct Range {
   uintptr_t lo, hi;  // [lo, hi)
@@ -65,7 +66,7 @@ float resolve_scale(const gdn_params_t* p) {
 
 }  // namespace
 
-GDN_API int gdn_version(void) { return (1 << 16) | 0; }
+GDN_API int gdn_version(void) { return (1 << 16) | 1; }
 
 GDN_API const char* gdn_status_string(int status) {
   switch (status) {
@@ -81,14 +82,18 @@ GDN_API const char* gdn_status_string(int status) {
   }
 }
 
-GDN_API int gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
-                          const float* beta, const float* initial_state,
-                          const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens,
-                          int32_t chunk_size, void* out, float* final_state,
+// Shared by gdn_chunk_fwd (A_log == dt_bias == nullptr: g and beta given) and
+// gdn_chunk_fwd_gated (g, beta slots hold the raw projections a, b).
+static int chunk_fwd_impl(const void* q, const void* k, const void* v, const float* g,
+                          const float* beta, const float* A_log, const float* dt_bias,
+                          const float* initial_state, const int32_t* cu_seqlens, int32_t num_seqs,
+                          int64_t total_tokens, int32_t chunk_size, void* out, float* final_state,
                           const gdn_params_t* p, void* cuda_stream) {
   int rc = check_params(p);
   if (rc) return rc;
   if (!q || !k || !v || !g || !beta || !out) return GDN_ERR_NULL;
+  if ((A_log == nullptr) != (dt_bias == nullptr)) return GDN_ERR_NULL;
+  if ((A_log && !aligned4(A_log)) || (dt_bias && !aligned4(dt_bias))) return GDN_ERR_ALIGN;
   if (num_seqs < 1 || num_seqs > 65535) return GDN_ERR_SHAPE;
   if (total_tokens < 0 || total_tokens >= (int64_t(1) << 31)) return GDN_ERR_SHAPE;
   if (chunk_size != 64 && chunk_size != 128) return GDN_ERR_SHAPE;
@@ -104,13 +109,15 @@ GDN_API int gdn_chunk_fwd(const void* q, const void* k, const void* v, const flo
   const Range rq = range_of(q, T * nqk * dk * esz), rk = range_of(k, T * nqk * dk * esz);
   const Range rv = range_of(v, T * nv * dv * esz);
   const Range rg = range_of(g, T * nv * 4), rb = range_of(beta, T * nv * 4);
+  const Range ra = A_log ? range_of(A_log, nv * 4) : Range{0, 0};
+  const Range rd = dt_bias ? range_of(dt_bias, nv * 4) : Range{0, 0};
   const Range rs0 = initial_state ? range_of(initial_state, N * nv * dk * dv * 4) : Range{0, 0};
   const Range rcu = cu_seqlens ? range_of(cu_seqlens, (N + 1) * 4) : Range{0, 0};
   const Range ro = range_of(out, T * nv * dv * esz);
   const Range rsf = final_state ? range_of(final_state, N * nv * dk * dv * 4) : Range{0, 0};
-  for (Range r : {rq, rk, rv, rg, rb, rs0, rcu, rsf})
+  for (Range r : {rq, rk, rv, rg, rb, ra, rd, rs0, rcu, rsf})
     if (overlap(ro, r)) return GDN_ERR_ALIAS;
-  for (Range r : {rq, rk, rv, rg, rb, rcu})
+  for (Range r : {rq, rk, rv, rg, rb, ra, rd, rcu})
     if (overlap(rsf, r)) return GDN_ERR_ALIAS;
   if (final_state && initial_state && (const void*)final_state != (const void*)initial_state &&
       overlap(rsf, rs0))
@@ -119,8 +126,8 @@ GDN_API int gdn_chunk_fwd(const void* q, const void* k, const void* v, const flo
   rc = check_device();
   if (rc) return rc;
 
-  gdn::ChunkArgs a;
-  a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta;
+  gdn::ChunkArgs a{};
+  a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.A_log = A_log; a.dt_bias = dt_bias;
   a.s0 = initial_state; a.cu = cu_seqlens; a.out = out; a.s_final = final_state;
   a.uniform_len = cu_seqlens ? 0 : (int32_t)(total_tokens / num_seqs);
   a.num_seqs = num_seqs;
@@ -140,12 +147,35 @@ GDN_API int gdn_chunk_fwd(const void* q, const void* k, const void* v, const flo
   return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
-GDN_API int gdn_recurrent_step(const void* q, const void* k, const void* v, const float* g,
-                               const float* beta, float* state, void* out, int32_t num_seqs,
-                               const gdn_params_t* p, void* cuda_stream) {
+GDN_API int gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
+                          const float* beta, const float* initial_state,
+                          const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                          int32_t chunk_size, void* out, float* final_state,
+                          const gdn_params_t* p, void* cuda_stream) {
+  return chunk_fwd_impl(q, k, v, g, beta, nullptr, nullptr, initial_state, cu_seqlens, num_seqs,
+                        total_tokens, chunk_size, out, final_state, p, cuda_stream);
+}
+
+GDN_API int gdn_chunk_fwd_gated(const void* q, const void* k, const void* v, const float* a,
+                                const float* b, const float* A_log, const float* dt_bias,
+                                const float* initial_state, const int32_t* cu_seqlens,
+                                int32_t num_seqs, int64_t total_tokens, int32_t chunk_size,
+                                void* out, float* final_state, const gdn_params_t* p,
+                                void* cuda_stream) {
+  if (!A_log || !dt_bias) return GDN_ERR_NULL;
+  return chunk_fwd_impl(q, k, v, a, b, A_log, dt_bias, initial_state, cu_seqlens, num_seqs,
+                        total_tokens, chunk_size, out, final_state, p, cuda_stream);
+}
+
+static int recurrent_step_impl(const void* q, const void* k, const void* v, const float* g,
+                               const float* beta, const float* A_log, const float* dt_bias,
+                               float* state, void* out, int32_t num_seqs, const gdn_params_t* p,
+                               void* cuda_stream) {
   int rc = check_params(p);
   if (rc) return rc;
   if (!q || !k || !v || !g || !beta || !state || !out) return GDN_ERR_NULL;
+  if ((A_log == nullptr) != (dt_bias == nullptr)) return GDN_ERR_NULL;
+  if ((A_log && !aligned4(A_log)) || (dt_bias && !aligned4(dt_bias))) return GDN_ERR_ALIGN;
   if (num_seqs < 1 || num_seqs > 65535) return GDN_ERR_SHAPE;
   const void* ptrs[] = {q, k, v, g, beta, state, out};
   for (const void* ptr : ptrs)
@@ -157,18 +187,21 @@ GDN_API int gdn_recurrent_step(const void* q, const void* k, const void* v, cons
   const Range rq = range_of(q, N * nqk * dk * esz), rk = range_of(k, N * nqk * dk * esz);
   const Range rv = range_of(v, N * nv * dv * esz);
   const Range rg = range_of(g, N * nv * 4), rb = range_of(beta, N * nv * 4);
+  const Range ra = A_log ? range_of(A_log, nv * 4) : Range{0, 0};
+  const Range rd = dt_bias ? range_of(dt_bias, nv * 4) : Range{0, 0};
   const Range rs = range_of(state, N * nv * dk * dv * 4);
   const Range ro = range_of(out, N * nv * dv * esz);
-  for (Range r : {rq, rk, rv, rg, rb, rs})
+  for (Range r : {rq, rk, rv, rg, rb, ra, rd, rs})
     if (overlap(ro, r)) return GDN_ERR_ALIAS;
-  for (Range r : {rq, rk, rv, rg, rb})
+  for (Range r : {rq, rk, rv, rg, rb, ra, rd})
     if (overlap(rs, r)) return GDN_ERR_ALIAS;
 
   rc = check_device();
   if (rc) return rc;
 
-  gdn::StepArgs a;
-  a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.state = state; a.out = out;
+  gdn::StepArgs a{};
+  a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.A_log = A_log; a.dt_bias = dt_bias;
+  a.state = state; a.out = out;
   a.num_seqs = num_seqs;
   a.nqk = p->num_qk_heads; a.nv = p->num_v_heads;
   a.qk_l2norm = p->qk_l2norm ? 1 : 0;
@@ -177,6 +210,20 @@ GDN_API int gdn_recurrent_step(const void* q, const void* k, const void* v, cons
                                              p->io_dtype == GDN_DTYPE_BF16,
                                              static_cast<cudaStream_t>(cuda_stream));
   return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+GDN_API int gdn_recurrent_step(const void* q, const void* k, const void* v, const float* g,
+                               const float* beta, float* state, void* out, int32_t num_seqs,
+                               const gdn_params_t* p, void* cuda_stream) {
+  return recurrent_step_impl(q, k, v, g, beta, nullptr, nullptr, state, out, num_seqs, p, cuda_stream);
+}
+
+GDN_API int gdn_recurrent_step_gated(const void* q, const void* k, const void* v, const float* a,
+                                     const float* b, const float* A_log, const float* dt_bias,
+                                     float* state, void* out, int32_t num_seqs,
+                                     const gdn_params_t* p, void* cuda_stream) {
+  if (!A_log || !dt_bias) return GDN_ERR_NULL;
+  return recurrent_step_impl(q, k, v, a, b, A_log, dt_bias, state, out, num_seqs, p, cuda_stream);
 }
 
 GDN_API int gdn_device_status(void* cuda_stream) {

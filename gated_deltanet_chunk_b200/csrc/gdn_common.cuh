@@ -15,8 +15,10 @@ struct ChunkArgs {
   const void* q;             // [T, Nqk, Dk]
   const void* k;             // [T, Nqk, Dk]
   const void* v;             // [T, Nv, Dv]
-  const float* g;            // [T, Nv]
-  const float* beta;         // [T, Nv]
+  const float* g;            // [T, Nv]: g, or the raw projection a when A_log != nullptr
+  const float* beta;         // [T, Nv]: beta, or the raw projection b when A_log != nullptr
+  const float* A_log;        // [Nv] or nullptr (g and beta given)
+  const float* dt_bias;      // [Nv] (used with A_log)
   const float* s0;           // [N, Nv, Dk, Dv] or nullptr
   const int32_t* cu;         // [N + 1] or nullptr (equal lengths)
   void* out;                 // [T, Nv, Dv]
@@ -33,8 +35,10 @@ struct StepArgs {
   const void* q;     // [N, Nqk, Dk]
   const void* k;     // [N, Nqk, Dk]
   const void* v;     // [N, Nv, Dv]
-  const float* g;    // [N, Nv]
-  const float* beta; // [N, Nv]
+  const float* g;    // [N, Nv]: g, or the raw projection a when A_log != nullptr
+  const float* beta; // [N, Nv]: beta, or the raw projection b when A_log != nullptr
+  const float* A_log;    // [Nv] or nullptr (g and beta given)
+  const float* dt_bias;  // [Nv] (used with A_log)
   float* state;      // [N, Nv, Dk, Dv] in place
   void* out;         // [N, Nv, Dv]
   int32_t num_seqs;
@@ -59,6 +63,25 @@ __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
   return x;
+}
+
+// The gate of row i (a token, or a sequence in a decode step) on v-head h.
+// Without A_log the caller passed g and beta.  With it, the g / beta slots hold
+// the layer's raw projections a and b, and the gate is formed as in the
+// "手撕Qwen3-Next" walkthrough, section 一(一)4:
+//   beta = sigmoid(b),  g = -exp(A_log[h]) * softplus(a + dt_bias[h]),
+// softplus(x) = log(1 + exp(x)), evaluated as max(x, 0) + log1p(exp(-|x|)).
+template <class Args>
+__device__ __forceinline__ void load_gate(const Args& a, size_t i, int h, float& g, float& beta) {
+  const float x = a.g[i], y = a.beta[i];
+  if (a.A_log == nullptr) {
+    g = x;
+    beta = y;
+    return;
+  }
+  const float u = x + a.dt_bias[h];
+  g = -expf(a.A_log[h]) * (fmaxf(u, 0.f) + log1pf(expf(-fabsf(u))));
+  beta = 1.f / (1.f + expf(-y));
 }
 
 // Sequence bounds [start, end) of sequence n.

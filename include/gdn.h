@@ -124,6 +124,38 @@ int gdn_recurrent_step(const void *q, const void *k, const void *v,
                        const gdn_params_t *p, void *cuda_stream);
 
 /*
+ * gdn_chunk_fwd_gated / gdn_recurrent_step_gated -- the same two calls with the
+ * gate formed in-kernel from the layer's raw projections, as in the walkthrough's
+ * section 一(一)4 (形状调整):
+ *
+ *   beta = sigmoid(b),   g = -exp(A_log[h]) * softplus(a + dt_bias[h]),
+ *   softplus(x) = log(1 + exp(x))   (evaluated as max(x,0) + log1p(exp(-|x|)))
+ *
+ *   a, b      [T, Nv] (prefill) or [N, Nv] (decode), fp32: take the places of g, beta
+ *   A_log     [Nv] fp32, the log of the per-head decay rate A > 0
+ *   dt_bias   [Nv] fp32
+ *
+ * A_log and dt_bias must be non-NULL and 4-byte aligned; every other argument,
+ * shape rule, overlap rule and status code is that of gdn_chunk_fwd /
+ * gdn_recurrent_step (a, b, A_log, dt_bias count as inputs).  The gate is
+ * evaluated in fp32 with the accurate CUDA expf / log1pf.
+ */
+int gdn_chunk_fwd_gated(const void *q, const void *k, const void *v,
+                        const float *a, const float *b,
+                        const float *A_log, const float *dt_bias,
+                        const float *initial_state,
+                        const int32_t *cu_seqlens,
+                        int32_t num_seqs, int64_t total_tokens, int32_t chunk_size,
+                        void *out, float *final_state,
+                        const gdn_params_t *p, void *cuda_stream);
+
+int gdn_recurrent_step_gated(const void *q, const void *k, const void *v,
+                             const float *a, const float *b,
+                             const float *A_log, const float *dt_bias,
+                             float *state, void *out, int32_t num_seqs,
+                             const gdn_params_t *p, void *cuda_stream);
+
+/*
  * gdn_device_status -- synchronise `cuda_stream`, then read and clear the
  * library's device-side error word for the current device.  Returns GDN_OK,
  * GDN_ERR_DEVICE_TIMEOUT if a kernel gave up a bounded wait since the last

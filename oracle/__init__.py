@@ -14,6 +14,8 @@ This module only marshals arrays:
 * :func:`chunk_form` -- the same walkthrough's chunkwise algorithm, section
   5(1) steps a-g, with a generic chunk size.  Used only to pin the two forms
   against each other.
+* :func:`gates` -- the layer's gate parametrisation (same walkthrough, section
+  4): beta = sigmoid(b), g = -exp(A_log) softplus(a + dt_bias).
 * :func:`chunk_prepare` -- the intra-chunk quantities of one chunk (gate
   cumsum, decay mask, A, T = (I - A)^-1, U, W), for the inverse and similarity
   pins.
@@ -67,6 +69,7 @@ def _load():
                                           ctypes.c_double, dp, dp]
         lib.oracle_chunk_form.restype = i
         lib.oracle_chunk_prepare.argtypes = [i, i, i, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp]
+        lib.oracle_gates.argtypes = [ctypes.c_int64, i, dp, dp, dp, dp, dp, dp]
         lib.oracle_chunk_prepare.restype = i
         _lib = lib
     return _lib
@@ -168,3 +171,23 @@ def num_threads() -> int:
         return len(os.sched_getaffinity(0))
     except AttributeError:  # pragma: no cover
         return os.cpu_count() or 1
+
+
+def gates(a, b, A_log, dt_bias):
+    """beta = sigmoid(b), g = -exp(A_log) softplus(a + dt_bias) in fp64 (oracle_gates).
+
+    ``a``, ``b`` are [..., Nv]; ``A_log``, ``dt_bias`` are [Nv].  Returns (g, beta)
+    as float64 numpy arrays of the shape of ``a``.
+    """
+    a64, b64 = _f64(a), _f64(b)
+    al, db = _f64(A_log).reshape(-1), _f64(dt_bias).reshape(-1)
+    nv = al.shape[0]
+    if a64.shape != b64.shape or a64.shape[-1] != nv or db.shape[0] != nv:
+        raise ValueError("gates: a, b [..., Nv] and A_log, dt_bias [Nv] expected")
+    T = a64.size // nv
+    g = np.empty_like(a64)
+    beta = np.empty_like(a64)
+    rc = _load().oracle_gates(T, nv, _ptr(a64), _ptr(b64), _ptr(al), _ptr(db), _ptr(g), _ptr(beta))
+    if rc != 0:
+        raise ValueError("oracle_gates failed (%d)" % rc)
+    return g, beta

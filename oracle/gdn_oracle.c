@@ -15,6 +15,12 @@
  *   [PTO] PyPTO-Gym "Qwen3Next 样例" README, sections 数学公式 (formulas) and
  *         参数说明 (packed [T,N,D] tensors, act_seq_len cumulative lengths).
  *
+ * Gate parametrisation ([WT] section 一(一)4 "形状调整", the lines that form
+ * beta and g from the projections b and a):
+ *
+ *   oracle_gates       -- beta = sigmoid(b);  g = -exp(A_log) * softplus(a + dt_bias)
+ *                         with softplus(x) = log(1 + exp(x)), per token and v-head.
+ *
  * Two functions compute the method:
  *
  *   oracle_recurrent   -- THE DEFINITION.  Token loop of [WT] (2):
@@ -316,6 +322,26 @@ int oracle_chunk_form(int num_seqs, const int32_t *cu_seqlens,
         if (s_final) memcpy(s_final + sidx, S, sizeof(double) * (size_t)dk * dv);
         free(Q); free(K); free(V); free(G); free(B); free(GC); free(GM); free(Am); free(Tm);
         free(U); free(W); free(S); free(Vn); free(P);
+    }
+    return 0;
+}
+
+/* Gate parametrisation, [WT] 一(一)4: beta = sigmoid(b), g = -exp(A_log) *
+ * softplus(a + dt_bias), softplus(x) = log(1 + exp(x)).  a, b, g, beta are
+ * [T, nv]; A_log, dt_bias are [nv].  softplus is evaluated as
+ * max(x, 0) + log1p(exp(-|x|)), the same function without overflow. */
+int oracle_gates(int64_t T, int nv, const double *a, const double *b, const double *A_log,
+                 const double *dt_bias, double *g, double *beta)
+{
+    if (T < 0 || nv <= 0 || !a || !b || !A_log || !dt_bias || !g || !beta) return -1;
+    for (int64_t t = 0; t < T; ++t) {
+        for (int h = 0; h < nv; ++h) {
+            const int64_t i = t * nv + h;
+            const double x = a[i] + dt_bias[h];
+            const double sp = (x > 0.0 ? x : 0.0) + log1p(exp(-fabs(x)));
+            g[i] = -exp(A_log[h]) * sp;
+            beta[i] = 1.0 / (1.0 + exp(-b[i]));
+        }
     }
     return 0;
 }

@@ -313,6 +313,45 @@ def pin_inverse_and_similarity():
     assert rel(r["T"], np.linalg.inv(I + L)) < 1e-10
 
 
+def pin_gates_closed_forms():
+    """Gate parametrisation (walkthrough section 4): beta = sigmoid(b),
+    g = -exp(A_log) softplus(a + dt_bias), softplus(x) = log(1 + exp(x)).
+
+    Pinned by values the definitions fix: sigmoid(0) = 1/2 and
+    sigmoid(x) + sigmoid(-x) = 1; softplus(0) = ln 2, softplus(x) - softplus(-x) = x,
+    d softplus/dx = sigmoid(x), softplus(x) ~ x for large x and ~ e^x for very
+    negative x; A_log and dt_bias are per v-head; g <= 0.
+    """
+    nv = 3
+    A = np.array([3.0, 0.5, 7.0])
+    A_log, db = np.log(A), np.array([1.0, -0.25, 2.0])
+    # a + dt_bias = 0 and b = 0 on every head
+    g, beta = oracle.gates(np.tile(-db, (2, 1)), np.zeros((2, nv)), A_log, db)
+    assert np.all(beta == 0.5)
+    assert np.max(np.abs(g - (-A * np.log(2.0)))) < 1e-15
+    # odd part of softplus and the sigmoid symmetry, on a grid of x = a + dt_bias
+    xs = np.linspace(-30.0, 30.0, 121)
+    a_p = xs[:, None] - db[None, :]
+    a_m = -xs[:, None] - db[None, :]
+    bb = np.repeat(xs[:, None], nv, axis=1)
+    gp, bp = oracle.gates(a_p, bb, A_log, db)
+    gm, bm = oracle.gates(a_m, -bb, A_log, db)
+    sp, sm = gp / -A, gm / -A
+    assert np.max(np.abs((sp - sm) - xs[:, None])) < 1e-12
+    assert np.max(np.abs(bp + bm - 1.0)) < 1e-15
+    assert np.all(gp <= 0.0) and np.all(gm <= 0.0)
+    # derivative of softplus is the sigmoid of the same argument
+    h = 1e-5
+    g1, _ = oracle.gates(a_p + h, bb, A_log, db)
+    g0, _ = oracle.gates(a_p - h, bb, A_log, db)
+    dsp = (g1 - g0) / (-A) / (2 * h)
+    assert np.max(np.abs(dsp - bp)) < 1e-8
+    # tails
+    gt, _ = oracle.gates(np.array([[40.0 - db[0], -40.0 - db[1], 0.0]]), np.zeros((1, nv)), A_log, db)
+    assert abs(gt[0, 0] / -A[0] - 40.0) < 1e-13
+    assert abs(gt[0, 1] / -A[1] / np.exp(-40.0) - 1.0) < 1e-12
+
+
 # --------------------------------------------------------------------------
 # Stored golden values (tests/golden/*.txt): outputs of small cases written by
 # tests/golden/make_golden.py from the oracle, so a later change of the oracle's
@@ -323,5 +362,5 @@ ALL_PINS = [
     pin_matrix_form, pin_l2norm_eps_closed_form, pin_scale_and_norm_invariance,
     pin_chunk_equals_recurrent, pin_beta_zero, pin_delta_write_exact, pin_zero_pad_invariance,
     pin_split_carry_and_varlen, pin_gqa_repeat_interleave, pin_linearity, pin_orthonormal_keys,
-    pin_dv_columns_independent, pin_inverse_and_similarity,
+    pin_dv_columns_independent, pin_inverse_and_similarity, pin_gates_closed_forms,
 ]

@@ -111,3 +111,25 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(g, "_lib", None)
     with pytest.raises(ImportError):
         g.lib()
+
+
+def _chunk_gated(L, p, al=A + 0x8000000, db=A + 0x8001000, out=A + 0x5000000):
+    vp = ctypes.c_void_p
+    return L.gdn_chunk_fwd_gated(vp(A), vp(A + 0x1000000), vp(A + 0x2000000), vp(A + 0x3000000),
+                                 vp(A + 0x4000000), vp(al), vp(db), None, None, 2, 256, 64, vp(out),
+                                 None, ctypes.byref(p), None)
+
+
+def test_gated_validation(L):
+    p = _p()
+    assert _chunk_gated(L, p, al=None) == -1            # A_log and dt_bias are required
+    assert _chunk_gated(L, p, db=None) == -1
+    assert _chunk_gated(L, p, al=A + 0x8000002) == -3   # 4-byte alignment
+    assert _chunk_gated(L, p, out=A + 0x8000000) == -4  # out over A_log
+    vp = ctypes.c_void_p
+    assert L.gdn_recurrent_step_gated(vp(A), vp(A + 0x100000), vp(A + 0x200000), vp(A + 0x300000),
+                                      vp(A + 0x400000), None, vp(A + 0x500000), vp(A + 0x600000),
+                                      vp(A + 0x900000), 4, ctypes.byref(p), None) == -1
+    import torch
+    if not torch.cuda.is_available():
+        assert _chunk_gated(L, p) in (-5, -6)          # valid: stops at the device check

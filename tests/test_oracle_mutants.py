@@ -19,6 +19,10 @@ SRC = os.path.join(ROOT, "oracle", "gdn_oracle.c")
 
 # (name, text to find, replacement, which occurrence (0-based))
 MUTANTS = [
+    ("gate_sign", "g[i] = -exp(A_log[h]) * sp;", "g[i] = exp(A_log[h]) * sp;", 0),
+    ("softplus_as_exp", "(x > 0.0 ? x : 0.0) + log1p(exp(-fabs(x)))", "exp(x)", 0),
+    ("sigmoid_sign", "beta[i] = 1.0 / (1.0 + exp(-b[i]));", "beta[i] = 1.0 / (1.0 + exp(b[i]));", 0),
+    ("gate_no_bias", "const double x = a[i] + dt_bias[h];", "const double x = a[i];", 0),
     ("no_decay", "S[e] *= alpha;", "S[e] *= 1.0;", 0),
     ("delta_sign", "kv[c] = b * (vt[c] - kv[c]);", "kv[c] = b * (vt[c] + kv[c]);", 0),
     ("kv_uses_query", "kv[c] += S[(size_t)r * dv + c] * kh[r];",

@@ -102,7 +102,9 @@ def make_prefill(num_seqs: int = 1, seq_len: Optional[int] = 256, nqk: int = 1, 
 
     Returns a dict with q, k [T,Nqk,Dk], v [T,Nv,Dv] (``io`` dtype), g, beta
     [T,Nv] fp32, initial_state [N,Nv,Dk,Dv] fp32 or None, cu_seqlens int32
-    [N+1], and the integer sizes.
+    [N+1], the integer sizes, and the raw gate inputs they were drawn from:
+    a, b [T,Nv] fp32, A_log = log A [Nv] and dt_bias [Nv] (= 1) fp32 (the
+    "gate" overrides above apply to g and beta only).
     """
     dv = d if dv is None else dv
     gen = torch.Generator(device="cpu").manual_seed(int(seed))
@@ -131,9 +133,12 @@ def make_prefill(num_seqs: int = 1, seq_len: Optional[int] = 256, nqk: int = 1, 
     if gate == "beta0":
         beta = torch.zeros_like(beta)
     out = dict(q=q, k=k, v=v, g=g, beta=beta, initial_state=s0, cu_seqlens=cu,
-               T=T, num_seqs=len(lengths), nqk=nqk, nv=nv, dk=d, dv=dv, io=io)
+               T=T, num_seqs=len(lengths), nqk=nqk, nv=nv, dk=d, dv=dv, io=io,
+               a=a.contiguous(), b=b.contiguous(), A_log=torch.log(A.float()).contiguous(),
+               dt_bias=torch.full((nv,), 1.0))
     if device != "cpu":
-        for key in ("q", "k", "v", "g", "beta", "initial_state", "cu_seqlens"):
+        for key in ("q", "k", "v", "g", "beta", "initial_state", "cu_seqlens", "a", "b", "A_log",
+                    "dt_bias"):
             if out[key] is not None:
                 out[key] = out[key].to(device)
     return out
@@ -157,7 +162,8 @@ def make_decode(num_seqs: int = 256, steps: int = 8, nqk: int = 16, nv: int = 32
     """Draw a decode run: ``steps`` fresh tokens for each of ``num_seqs`` sequences.
 
     Returns q, k [steps,N,Nqk,D], v [steps,N,Nv,D] (``io`` dtype), g, beta
-    [steps,N,Nv] fp32 and the initial state [N,Nv,D,D] fp32.  Drawn on
+    [steps,N,Nv] fp32, the initial state [N,Nv,D,D] fp32, and the raw gate
+    inputs a, b [steps,N,Nv], A_log [Nv], dt_bias [Nv] (= 1) fp32.  Drawn on
     ``device`` with a generator of that device (CPU and CUDA streams differ).
     """
     gen = torch.Generator(device=device).manual_seed(int(seed))
@@ -172,4 +178,6 @@ def make_decode(num_seqs: int = 256, steps: int = 8, nqk: int = 16, nv: int = 32
     s0 = torch.randn(num_seqs, nv, d, d, **kw) * state_std
     g, beta = draw_gates(b, a, A)
     return dict(q=q, k=k, v=v, g=g, beta=beta, initial_state=s0, num_seqs=num_seqs,
-                steps=steps, nqk=nqk, nv=nv, dk=d, dv=d, io=io)
+                steps=steps, nqk=nqk, nv=nv, dk=d, dv=d, io=io,
+                a=a.contiguous(), b=b.contiguous(), A_log=torch.log(A.float()).contiguous(),
+                dt_bias=torch.full((nv,), 1.0, device=device))
