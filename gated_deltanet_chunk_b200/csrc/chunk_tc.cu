@@ -167,6 +167,7 @@ __device__ __forceinline__ bool named_bar_any(int id, int nthreads, bool flag) {
 }
 
 
+template <bool kRawGate>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const ChunkArgs a) {
@@ -247,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     {
       const int64_t t0g = seq_start + (int64_t)crank * C + t;
       if (t < 64 && t0g < seq_end) {
-        load_gate(a, (size_t)t0g * nv + h, h, g_next, b_next);
+        load_gate_t<kRawGate>(a, (size_t)t0g * nv + h, h, g_next, b_next);
       }
     }
 
@@ -278,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         g_next = 0.f;
         b_next = 0.f;
         if (tn < seq_end) {
-          load_gate(a, (size_t)tn * nv + h, h, g_next, b_next);
+          load_gate_t<kRawGate>(a, (size_t)tn * nv + h, h, g_next, b_next);
         }
       }
       wait_bar(bars + BAR_RAWF + rsl, (uint32_t)((c / NR) & 1));
@@ -806,8 +807,9 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int64_t total_tokens, cudaStream
   if (!tc::make_map(&mq, a.q, a.nqk, total_tokens) || !tc::make_map(&mk, a.k, a.nqk, total_tokens) ||
       !tc::make_map(&mv, a.v, a.nv, total_tokens))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(tc::chunk_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       tc::SMEM_BYTES);
+  const bool raw_gate = a.A_log != nullptr;
+  auto kernel = raw_gate ? tc::chunk_fwd_tc_kernel<true> : tc::chunk_fwd_tc_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.dv / tc::DVS, a.nv, a.num_seqs);  // x: the two Dv slices = one cluster
@@ -821,7 +823,7 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int64_t total_tokens, cudaStream
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, tc::chunk_fwd_tc_kernel, mq, mk, mv, a);
+  e = cudaLaunchKernelEx(&cfg, kernel, mq, mk, mv, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

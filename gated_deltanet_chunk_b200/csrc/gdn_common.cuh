@@ -72,16 +72,29 @@ __device__ __forceinline__ float warp_sum(float x) {
 //   beta = sigmoid(b),  g = -exp(A_log[h]) * softplus(a + dt_bias[h]),
 // softplus(x) = log(1 + exp(x)), evaluated as max(x, 0) + log1p(exp(-|x|)).
 template <class Args>
-__device__ __forceinline__ void load_gate(const Args& a, size_t i, int h, float& g, float& beta) {
-  const float x = a.g[i], y = a.beta[i];
-  if (a.A_log == nullptr) {
-    g = x;
-    beta = y;
-    return;
-  }
-  const float u = x + a.dt_bias[h];
+__device__ __forceinline__ void gate_from_raw(const Args& a, size_t i, int h, float& g, float& beta) {
+  const float u = a.g[i] + a.dt_bias[h];
   g = -expf(a.A_log[h]) * (fmaxf(u, 0.f) + log1pf(expf(-fabsf(u))));
-  beta = 1.f / (1.f + expf(-y));
+  beta = 1.f / (1.f + expf(-a.beta[i]));
+}
+template <class Args>
+__device__ __forceinline__ void load_gate(const Args& a, size_t i, int h, float& g, float& beta) {
+  if (a.A_log == nullptr) {
+    g = a.g[i];
+    beta = a.beta[i];
+  } else {
+    gate_from_raw(a, i, h, g, beta);
+  }
+}
+// The same with the mode fixed at compile time (kernels instantiated per mode).
+template <bool kRaw, class Args>
+__device__ __forceinline__ void load_gate_t(const Args& a, size_t i, int h, float& g, float& beta) {
+  if constexpr (kRaw) {
+    gate_from_raw(a, i, h, g, beta);
+  } else {
+    g = a.g[i];
+    beta = a.beta[i];
+  }
 }
 
 // Sequence bounds [start, end) of sequence n.
