@@ -267,6 +267,35 @@ def run_ours(args, world, rank, local):
                                              fl_tri / (peaks["bf16_tflops"] * 1e12)) * 1e3},
         "clocks": clk.summary(),
     }
+    # the same workload with the gate formed in-kernel from the raw projections
+    if not args.no_gated:
+        ga = {k_: host[k_].to(dev) for k_ in ("a", "b", "A_log", "dt_bias")}
+
+        def gstep():
+            gdn.chunk_fwd_gated(d["q"], d["k"], d["v"], ga["a"], ga["b"], ga["A_log"], ga["dt_bias"],
+                                None, None, chunk_size=C, out=out, final_state=sf, num_seqs=n)
+
+        for _ in range(args.warmup):
+            gstep()
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a_.record(stream)
+        for _ in range(args.steps):
+            gstep()
+        b_.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        g_ms = max_over_ranks(a_.elapsed_time(b_), world, dev) / args.steps
+        g_bytes = bytes_alg + 2 * nv * 4  # a, b replace g, beta; plus A_log, dt_bias
+        res["gated"] = {"value": T * world / (g_ms / 1e3), "unit": "tokens/s", "ms_per_step": g_ms,
+                        "call": "gdn_chunk_fwd_gated", "gpu_launches": args.steps,
+                        "roofline": {"bound": "hbm", "achieved": g_bytes / (g_ms / 1e3) / 1e9,
+                                     "peak": peaks[peak_key], "unit": "GB/s",
+                                     "frac": g_bytes / (g_ms / 1e3) / 1e9 / peaks[peak_key],
+                                     "traffic": None, "peak_source": peak_src,
+                                     "alg_bytes_per_launch": g_bytes}}
+        del ga
     # e2e: same call with host buffers (pinned), copies inside the timed region
     if not args.no_e2e:
         hp = {k: host[k].pin_memory() for k in ("q", "k", "v", "g", "beta")}
@@ -341,12 +370,65 @@ def run_decode(args, world, rank, dev, stream, peaks, peak_src):
     per_step_ms = ms / steps
     byts = decode_bytes(wl.num_seqs, wl.nqk, wl.nv, wl.d, wl.d, 2)
     gbs = byts / (per_step_ms / 1e3) / 1e9
-    return {"value": wl.num_seqs * steps * world / (ms / 1e3), "unit": "tokens/s",
-            "workload": DECODE, "steps": steps, "ms_per_step": per_step_ms, "gpu_launches": steps,
-            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": gbs / peaks["hbm_gbs"], "traffic": recorded_traffic("recurrent_step", wl.num_seqs),
-                         "peak_source": peak_src,
-                         "alg_bytes_per_launch": byts}}
+    res = {"value": wl.num_seqs * steps * world / (ms / 1e3), "unit": "tokens/s",
+           "workload": DECODE, "steps": steps, "ms_per_step": per_step_ms, "gpu_launches": steps,
+           "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": gbs / peaks["hbm_gbs"], "traffic": recorded_traffic("recurrent_step", wl.num_seqs),
+                        "peak_source": peak_src,
+                        "alg_bytes_per_launch": byts}}
+    if not args.no_slots:
+        # the same decode with the states in a 2x larger pool, rows chosen by a permutation
+        P = 2 * wl.num_seqs
+        gen = torch.Generator(device="cpu").manual_seed(7)
+        ids = torch.randperm(P, generator=gen)[: wl.num_seqs].to(torch.int32).to(dev)
+        pool = torch.zeros(P, wl.nv, wl.d, wl.d, dtype=torch.float32, device=dev)
+        pool[ids.long()] = state
+
+        def run_slots(n_steps):
+            for t in range(n_steps):
+                gdn.recurrent_step_slots(d["q"][t], d["k"][t], d["v"][t], d["g"][t], d["beta"][t],
+                                         pool, ids, out=out)
+
+        run_slots(min(steps, 32))
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        a.record(stream)
+        run_slots(steps)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        sms = max_over_ranks(a.elapsed_time(b), world, dev) / steps
+        sb = byts + wl.num_seqs * 4
+        res["slots"] = {"ms_per_step": sms, "value": wl.num_seqs * world / (sms / 1e3), "unit": "tokens/s",
+                        "call": "gdn_recurrent_step_slots", "pool_rows": P, "gpu_launches": steps,
+                        "roofline": {"bound": "hbm", "achieved": sb / (sms / 1e3) / 1e9,
+                                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                     "frac": sb / (sms / 1e3) / 1e9 / peaks["hbm_gbs"], "traffic": None,
+                                     "peak_source": peak_src, "alg_bytes_per_launch": sb}}
+        del pool
+    if not args.no_gated:
+        def run_gated(n_steps):
+            for t in range(n_steps):
+                gdn.recurrent_step_gated(d["q"][t], d["k"][t], d["v"][t], d["a"][t], d["b"][t],
+                                         d["A_log"], d["dt_bias"], state, out=out)
+
+        run_gated(min(steps, 32))
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        a.record(stream)
+        run_gated(steps)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        gms = max_over_ranks(a.elapsed_time(b), world, dev) / steps
+        gb = byts + 2 * wl.nv * 4
+        res["gated"] = {"ms_per_step": gms, "value": wl.num_seqs * world / (gms / 1e3), "unit": "tokens/s",
+                        "call": "gdn_recurrent_step_gated", "gpu_launches": steps,
+                        "roofline": {"bound": "hbm", "achieved": gb / (gms / 1e3) / 1e9,
+                                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                     "frac": gb / (gms / 1e3) / 1e9 / peaks["hbm_gbs"], "traffic": None,
+                                     "peak_source": peak_src, "alg_bytes_per_launch": gb}}
+    return res
 
 
 def run_reference(args, world, rank):
@@ -394,6 +476,8 @@ def main():
     ap.add_argument("--kernel", choices=["auto", "simt", "tc"], default="auto",
                     help="prefill kernel selection passed to gdn_chunk_fwd (default: auto)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-gated", action="store_true", help="skip the fused-gate prefill and decode lines")
+    ap.add_argument("--no-slots", action="store_true", help="skip the slot-indexed decode line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=0,
                     help="oracle sample per sequence for cpu_baseline (default: the whole workload)")

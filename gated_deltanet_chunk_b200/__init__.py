@@ -66,6 +66,12 @@ def lib() -> ctypes.CDLL:
         L.gdn_recurrent_step_gated.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, vp, ctypes.c_int32,
                                                ctypes.POINTER(GdnParams), vp]
         L.gdn_recurrent_step_gated.restype = ctypes.c_int
+        L.gdn_chunk_fwd_slots.argtypes = [vp, vp, vp, fp, fp, fp, ip, ctypes.c_int32, ip, ctypes.c_int32,
+                                          ctypes.c_int64, ctypes.c_int32, vp, ctypes.POINTER(GdnParams), vp]
+        L.gdn_chunk_fwd_slots.restype = ctypes.c_int
+        L.gdn_recurrent_step_slots.argtypes = [vp, vp, vp, fp, fp, fp, ip, ctypes.c_int32, vp, ctypes.c_int32,
+                                               ctypes.POINTER(GdnParams), vp]
+        L.gdn_recurrent_step_slots.restype = ctypes.c_int
         L.gdn_device_status.argtypes = [vp]
         L.gdn_device_status.restype = ctypes.c_int
         L.gdn_status_string.argtypes = [ctypes.c_int]
@@ -177,3 +183,42 @@ def recurrent_step_gated(q, k, v, a, b, A_log, dt_bias, state, out=None, qk_l2no
 def device_status(stream=None) -> int:
     """Synchronise the stream and return the library's device status (``gdn_device_status``)."""
     return lib().gdn_device_status(_stream(stream))
+
+
+def chunk_fwd_slots(q, k, v, g, beta, state_pool, slot_ids, cu_seqlens=None, chunk_size=64, out=None,
+                    num_seqs=None, qk_l2norm=True, scale=0.0, kernel="auto", stream=None, check=True):
+    """Chunked forward with the states in a slot-indexed pool, updated in place (``gdn_chunk_fwd_slots``).
+
+    state_pool [P, Nv, Dk, Dv] fp32; slot_ids [N] int32 (ids outside [0, P) mark padding
+    sequences); cu_seqlens [N+1] or None.  Returns out [T, Nv, Dv].
+    """
+    import torch
+    T, nqk, dk = q.shape
+    nv, dv = v.shape[1], v.shape[2]
+    n = slot_ids.numel()
+    if out is None:
+        out = torch.empty((T, nv, dv), dtype=v.dtype, device=v.device)
+    p = make_params(nqk, nv, dk, dv, q.dtype == torch.bfloat16, qk_l2norm, scale, kernel)
+    rc = lib().gdn_chunk_fwd_slots(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_pool),
+                                   _ptr(slot_ids), int(state_pool.shape[0]), _ptr(cu_seqlens), int(n),
+                                   int(T), int(chunk_size), _ptr(out), ctypes.byref(p), _stream(stream))
+    if check and rc != GDN_OK:
+        raise GdnError(rc, "gdn_chunk_fwd_slots")
+    return out
+
+
+def recurrent_step_slots(q, k, v, g, beta, state_pool, slot_ids, out=None, qk_l2norm=True, scale=0.0,
+                         stream=None, check=True):
+    """One decode token per sequence with slot-indexed states (``gdn_recurrent_step_slots``)."""
+    import torch
+    N, nqk, dk = q.shape
+    nv, dv = v.shape[1], v.shape[2]
+    if out is None:
+        out = torch.empty((N, nv, dv), dtype=v.dtype, device=v.device)
+    p = make_params(nqk, nv, dk, dv, q.dtype == torch.bfloat16, qk_l2norm, scale)
+    rc = lib().gdn_recurrent_step_slots(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_pool),
+                                        _ptr(slot_ids), int(state_pool.shape[0]), _ptr(out), int(N),
+                                        ctypes.byref(p), _stream(stream))
+    if check and rc != GDN_OK:
+        raise GdnError(rc, "gdn_recurrent_step_slots")
+    return out

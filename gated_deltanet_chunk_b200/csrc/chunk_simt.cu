@@ -133,10 +133,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_simt_kernel(ChunkArgs a
   float* eg = sm + L::kEg;
   float* ekl = sm + L::kEkl;
 
-  const size_t state_off = ((size_t)n * nv + h) * (size_t)DK * dv;
+  const int64_t srow = state_row(a, n);  // -1: a padding sequence (zero state, nothing stored)
+  const size_t state_off = ((size_t)(srow < 0 ? 0 : srow) * nv + h) * (size_t)DK * dv;
   for (int e = tid; e < DK * kDVS; e += kThreads) {
     const int d = e / kDVS, c = e % kDVS;
-    S[e] = a.s0 ? a.s0[state_off + (size_t)d * dv + cslice + c] : 0.f;
+    S[e] = (a.s0 && srow >= 0) ? a.s0[state_off + (size_t)d * dv + cslice + c] : 0.f;
   }
 
   for (int64_t c0 = seq_start; c0 < seq_end; c0 += C) {
@@ -356,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_simt_kernel(ChunkArgs a
     }
   }
   __syncthreads();
-  if (a.s_final) {
+  if (a.s_final && srow >= 0) {
     for (int e = tid; e < DK * kDVS; e += kThreads) {
       const int d = e / kDVS, c = e % kDVS;
       a.s_final[state_off + (size_t)d * dv + cslice + c] = S[e];

@@ -535,11 +535,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // =====================================================================
     const int t = tid - 256;  // 0..127: row d of the state
     // S lives in TMEM (fp32) and, rounded to bf16, in shared memory
-    const size_t st_off = ((size_t)n * nv + h) * (size_t)DK * dv + (size_t)t * dv + slice * DVS;
+    const int64_t srow = state_row(a, n);  // -1: a padding sequence (zero state, nothing stored)
+    const size_t st_off = ((size_t)(srow < 0 ? 0 : srow) * nv + h) * (size_t)DK * dv + (size_t)t * dv + slice * DVS;
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
       float x[32];
-      if (a.s0) {
+      if (a.s0 && srow >= 0) {
         const float4* src = reinterpret_cast<const float4*>(a.s0 + st_off + 32 * hh);
 #pragma unroll
         for (int cc = 0; cc < 8; ++cc) {
@@ -746,7 +747,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int cn = consumed; cn < issued; ++cn)
         ptx::mbar_wait_bounded(bars + BAR_RAWF + cn % NR, (uint32_t)((cn / NR) & 1), kWaitNs);
     }
-    if (ok && a.s_final) {
+    if (ok && a.s_final && srow >= 0) {
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         float x[32];

@@ -40,7 +40,12 @@ __global__ void __launch_bounds__(kThreads, 2) recurrent_step_kernel(StepArgs a)
   const int j = h / (a.nv / a.nqk);
   const int cg = tid % CG, rg = tid / CG;
 
-  float4* st = reinterpret_cast<float4*>(a.state + ((size_t)n * a.nv + h) * (size_t)DK * DV);
+  const int64_t srow = state_row(a, n);
+  if (srow < 0) {  // a padding sequence: zero output, no state
+    for (int c = tid; c < DV; c += kThreads) static_cast<IO*>(a.out)[((size_t)n * a.nv + h) * DV + c] = from_f32<IO>(0.f);
+    return;
+  }
+  float4* st = reinterpret_cast<float4*>(a.state + ((size_t)srow * a.nv + h) * (size_t)DK * DV);
   float4 s[RPT];
 #pragma unroll
   for (int i = 0; i < RPT; ++i) s[i] = __ldcs(st + (size_t)(i * RG + rg) * CG + cg);

@@ -66,7 +66,7 @@ float resolve_scale(const gdn_params_t* p) {
 
 }  // namespace
 
-GDN_API int gdn_version(void) { return (1 << 16) | 1; }
+GDN_API int gdn_version(void) { return (1 << 16) | 2; }
 
 GDN_API const char* gdn_status_string(int status) {
   switch (status) {
@@ -88,7 +88,8 @@ static int chunk_fwd_impl(const void* q, const void* k, const void* v, const flo
                           const float* beta, const float* A_log, const float* dt_bias,
                           const float* initial_state, const int32_t* cu_seqlens, int32_t num_seqs,
                           int64_t total_tokens, int32_t chunk_size, void* out, float* final_state,
-                          const gdn_params_t* p, void* cuda_stream) {
+                          const gdn_params_t* p, void* cuda_stream, const int32_t* slots = nullptr,
+                          int32_t num_slots = 0) {
   int rc = check_params(p);
   if (rc) return rc;
   if (!q || !k || !v || !g || !beta || !out) return GDN_ERR_NULL;
@@ -111,13 +112,15 @@ static int chunk_fwd_impl(const void* q, const void* k, const void* v, const flo
   const Range rg = range_of(g, T * nv * 4), rb = range_of(beta, T * nv * 4);
   const Range ra = A_log ? range_of(A_log, nv * 4) : Range{0, 0};
   const Range rd = dt_bias ? range_of(dt_bias, nv * 4) : Range{0, 0};
-  const Range rs0 = initial_state ? range_of(initial_state, N * nv * dk * dv * 4) : Range{0, 0};
+  const size_t rows = slots ? (size_t)num_slots : N;  // state rows
+  const Range rs0 = initial_state ? range_of(initial_state, rows * nv * dk * dv * 4) : Range{0, 0};
   const Range rcu = cu_seqlens ? range_of(cu_seqlens, (N + 1) * 4) : Range{0, 0};
+  const Range rsl = slots ? range_of(slots, N * 4) : Range{0, 0};
   const Range ro = range_of(out, T * nv * dv * esz);
-  const Range rsf = final_state ? range_of(final_state, N * nv * dk * dv * 4) : Range{0, 0};
-  for (Range r : {rq, rk, rv, rg, rb, ra, rd, rs0, rcu, rsf})
+  const Range rsf = final_state ? range_of(final_state, rows * nv * dk * dv * 4) : Range{0, 0};
+  for (Range r : {rq, rk, rv, rg, rb, ra, rd, rs0, rcu, rsl, rsf})
     if (overlap(ro, r)) return GDN_ERR_ALIAS;
-  for (Range r : {rq, rk, rv, rg, rb, ra, rd, rcu})
+  for (Range r : {rq, rk, rv, rg, rb, ra, rd, rcu, rsl})
     if (overlap(rsf, r)) return GDN_ERR_ALIAS;
   if (final_state && initial_state && (const void*)final_state != (const void*)initial_state &&
       overlap(rsf, rs0))
@@ -129,6 +132,7 @@ static int chunk_fwd_impl(const void* q, const void* k, const void* v, const flo
   gdn::ChunkArgs a{};
   a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.A_log = A_log; a.dt_bias = dt_bias;
   a.s0 = initial_state; a.cu = cu_seqlens; a.out = out; a.s_final = final_state;
+  a.slots = slots; a.num_slots = num_slots;
   a.uniform_len = cu_seqlens ? 0 : (int32_t)(total_tokens / num_seqs);
   a.num_seqs = num_seqs;
   a.nqk = p->num_qk_heads; a.nv = p->num_v_heads; a.dv = p->head_v_dim;
@@ -156,6 +160,18 @@ GDN_API int gdn_chunk_fwd(const void* q, const void* k, const void* v, const flo
                         total_tokens, chunk_size, out, final_state, p, cuda_stream);
 }
 
+GDN_API int gdn_chunk_fwd_slots(const void* q, const void* k, const void* v, const float* g,
+                                const float* beta, float* state_pool, const int32_t* slot_ids,
+                                int32_t num_slots, const int32_t* cu_seqlens, int32_t num_seqs,
+                                int64_t total_tokens, int32_t chunk_size, void* out,
+                                const gdn_params_t* p, void* cuda_stream) {
+  if (!state_pool || !slot_ids) return GDN_ERR_NULL;
+  if (num_slots < 1) return GDN_ERR_SHAPE;
+  if (!aligned4(slot_ids)) return GDN_ERR_ALIGN;
+  return chunk_fwd_impl(q, k, v, g, beta, nullptr, nullptr, state_pool, cu_seqlens, num_seqs,
+                        total_tokens, chunk_size, out, state_pool, p, cuda_stream, slot_ids, num_slots);
+}
+
 GDN_API int gdn_chunk_fwd_gated(const void* q, const void* k, const void* v, const float* a,
                                 const float* b, const float* A_log, const float* dt_bias,
                                 const float* initial_state, const int32_t* cu_seqlens,
@@ -170,7 +186,8 @@ GDN_API int gdn_chunk_fwd_gated(const void* q, const void* k, const void* v, con
 static int recurrent_step_impl(const void* q, const void* k, const void* v, const float* g,
                                const float* beta, const float* A_log, const float* dt_bias,
                                float* state, void* out, int32_t num_seqs, const gdn_params_t* p,
-                               void* cuda_stream) {
+                               void* cuda_stream, const int32_t* slots = nullptr,
+                               int32_t num_slots = 0) {
   int rc = check_params(p);
   if (rc) return rc;
   if (!q || !k || !v || !g || !beta || !state || !out) return GDN_ERR_NULL;
@@ -189,11 +206,12 @@ static int recurrent_step_impl(const void* q, const void* k, const void* v, cons
   const Range rg = range_of(g, N * nv * 4), rb = range_of(beta, N * nv * 4);
   const Range ra = A_log ? range_of(A_log, nv * 4) : Range{0, 0};
   const Range rd = dt_bias ? range_of(dt_bias, nv * 4) : Range{0, 0};
-  const Range rs = range_of(state, N * nv * dk * dv * 4);
+  const Range rs = range_of(state, (slots ? (size_t)num_slots : N) * nv * dk * dv * 4);
+  const Range rsl = slots ? range_of(slots, N * 4) : Range{0, 0};
   const Range ro = range_of(out, N * nv * dv * esz);
-  for (Range r : {rq, rk, rv, rg, rb, ra, rd, rs})
+  for (Range r : {rq, rk, rv, rg, rb, ra, rd, rs, rsl})
     if (overlap(ro, r)) return GDN_ERR_ALIAS;
-  for (Range r : {rq, rk, rv, rg, rb, ra, rd})
+  for (Range r : {rq, rk, rv, rg, rb, ra, rd, rsl})
     if (overlap(rs, r)) return GDN_ERR_ALIAS;
 
   rc = check_device();
@@ -201,7 +219,7 @@ static int recurrent_step_impl(const void* q, const void* k, const void* v, cons
 
   gdn::StepArgs a{};
   a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.A_log = A_log; a.dt_bias = dt_bias;
-  a.state = state; a.out = out;
+  a.state = state; a.out = out; a.slots = slots; a.num_slots = num_slots;
   a.num_seqs = num_seqs;
   a.nqk = p->num_qk_heads; a.nv = p->num_v_heads;
   a.qk_l2norm = p->qk_l2norm ? 1 : 0;
@@ -216,6 +234,17 @@ GDN_API int gdn_recurrent_step(const void* q, const void* k, const void* v, cons
                                const float* beta, float* state, void* out, int32_t num_seqs,
                                const gdn_params_t* p, void* cuda_stream) {
   return recurrent_step_impl(q, k, v, g, beta, nullptr, nullptr, state, out, num_seqs, p, cuda_stream);
+}
+
+GDN_API int gdn_recurrent_step_slots(const void* q, const void* k, const void* v, const float* g,
+                                     const float* beta, float* state_pool, const int32_t* slot_ids,
+                                     int32_t num_slots, void* out, int32_t num_seqs,
+                                     const gdn_params_t* p, void* cuda_stream) {
+  if (!slot_ids) return GDN_ERR_NULL;
+  if (num_slots < 1) return GDN_ERR_SHAPE;
+  if (!aligned4(slot_ids)) return GDN_ERR_ALIGN;
+  return recurrent_step_impl(q, k, v, g, beta, nullptr, nullptr, state_pool, out, num_seqs, p,
+                             cuda_stream, slot_ids, num_slots);
 }
 
 GDN_API int gdn_recurrent_step_gated(const void* q, const void* k, const void* v, const float* a,

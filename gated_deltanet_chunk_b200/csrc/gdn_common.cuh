@@ -19,7 +19,9 @@ struct ChunkArgs {
   const float* beta;         // [T, Nv]: beta, or the raw projection b when A_log != nullptr
   const float* A_log;        // [Nv] or nullptr (g and beta given)
   const float* dt_bias;      // [Nv] (used with A_log)
-  const float* s0;           // [N, Nv, Dk, Dv] or nullptr
+  const float* s0;           // [N, Nv, Dk, Dv] (or [num_slots, ...] with slots) or nullptr
+  const int32_t* slots;      // [N] state row of each sequence, or nullptr (row n)
+  int32_t num_slots;         // rows of the state pool when slots != nullptr
   const int32_t* cu;         // [N + 1] or nullptr (equal lengths)
   void* out;                 // [T, Nv, Dv]
   float* s_final;            // [N, Nv, Dk, Dv] or nullptr
@@ -39,7 +41,9 @@ struct StepArgs {
   const float* beta; // [N, Nv]: beta, or the raw projection b when A_log != nullptr
   const float* A_log;    // [Nv] or nullptr (g and beta given)
   const float* dt_bias;  // [Nv] (used with A_log)
-  float* state;      // [N, Nv, Dk, Dv] in place
+  float* state;      // [N, Nv, Dk, Dv] (or [num_slots, ...] with slots) in place
+  const int32_t* slots;  // [N] state row of each sequence, or nullptr (row n)
+  int32_t num_slots;     // rows of the state pool when slots != nullptr
   void* out;         // [N, Nv, Dv]
   int32_t num_seqs;
   int32_t nqk, nv;
@@ -95,6 +99,16 @@ __device__ __forceinline__ void load_gate_t(const Args& a, size_t i, int h, floa
     g = a.g[i];
     beta = a.beta[i];
   }
+}
+
+// State row of sequence n: n, or slots[n] with a slot map.  An id outside
+// [0, num_slots) marks a padding sequence and gives -1 (no state is read or
+// written for it).
+template <class Args>
+__device__ __forceinline__ int64_t state_row(const Args& a, int n) {
+  if (a.slots == nullptr) return n;
+  const int32_t s = a.slots[n];
+  return (s >= 0 && s < a.num_slots) ? (int64_t)s : -1;
 }
 
 // Sequence bounds [start, end) of sequence n.

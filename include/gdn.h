@@ -124,6 +124,41 @@ int gdn_recurrent_step(const void *q, const void *k, const void *v,
                        const gdn_params_t *p, void *cuda_stream);
 
 /*
+ * gdn_chunk_fwd_slots / gdn_recurrent_step_slots -- the same two calls with the
+ * recurrent states kept in a pool of rows, as a serving cache holds them (the
+ * walkthrough's Cache section: one [Nv, Dk, Dv] recurrent state per sequence),
+ * addressed through per-sequence slot ids and updated in place:
+ *
+ *   state_pool  [num_slots, Nv, Dk, Dv] fp32: row slot_ids[n] is the state of
+ *               sequence n on entry and is overwritten with its state on exit
+ *   slot_ids    [N] int32 device array, 4-byte aligned.  An id outside
+ *               [0, num_slots) marks a padding sequence: it is processed from a
+ *               zero state and nothing is stored for it (gdn_recurrent_step_slots
+ *               writes zeros to its output row).  Active sequences must have
+ *               distinct ids; contents are not otherwise validated.
+ *   num_slots   >= 1
+ *
+ * gdn_chunk_fwd_slots with cu_seqlens advances every sequence by its own number
+ * of tokens (1 for a plain decode step, more for a multi-token step or a
+ * prefill into the cache); it always uses the chunked kernels.  The pool and
+ * the slot ids count as inputs for the overlap rules; the pool may not
+ * overlap out.  Other arguments and status codes are those of gdn_chunk_fwd /
+ * gdn_recurrent_step.
+ */
+int gdn_chunk_fwd_slots(const void *q, const void *k, const void *v,
+                        const float *g, const float *beta,
+                        float *state_pool, const int32_t *slot_ids, int32_t num_slots,
+                        const int32_t *cu_seqlens,
+                        int32_t num_seqs, int64_t total_tokens, int32_t chunk_size,
+                        void *out, const gdn_params_t *p, void *cuda_stream);
+
+int gdn_recurrent_step_slots(const void *q, const void *k, const void *v,
+                             const float *g, const float *beta,
+                             float *state_pool, const int32_t *slot_ids, int32_t num_slots,
+                             void *out, int32_t num_seqs,
+                             const gdn_params_t *p, void *cuda_stream);
+
+/*
  * gdn_chunk_fwd_gated / gdn_recurrent_step_gated -- the same two calls with the
  * gate formed in-kernel from the layer's raw projections, as in the walkthrough's
  * section 一(一)4 (形状调整):

@@ -133,3 +133,23 @@ def test_gated_validation(L):
     import torch
     if not torch.cuda.is_available():
         assert _chunk_gated(L, p) in (-5, -6)          # valid: stops at the device check
+
+
+def test_slots_validation(L):
+    vp, p = ctypes.c_void_p, _p()
+
+    def chunk(pool=A + 0x8000000, slots=A + 0x9000000, nslots=16, out=A + 0x5000000):
+        return L.gdn_chunk_fwd_slots(vp(A), vp(A + 0x1000000), vp(A + 0x2000000), vp(A + 0x3000000),
+                                     vp(A + 0x4000000), vp(pool), vp(slots), nslots, None, 2, 256, 64,
+                                     vp(out), ctypes.byref(p), None)
+    assert chunk(pool=None) == -1
+    assert chunk(slots=None) == -1
+    assert chunk(nslots=0) == -2
+    assert chunk(slots=A + 0x9000002) == -3          # 4-byte alignment of the slot ids
+    assert chunk(out=A + 0x8000000) == -4            # out over the pool
+    assert L.gdn_recurrent_step_slots(vp(A), vp(A + 0x100000), vp(A + 0x200000), vp(A + 0x300000),
+                                      vp(A + 0x400000), vp(A + 0x500000), None, 8, vp(A + 0x900000), 4,
+                                      ctypes.byref(p), None) == -1
+    import torch
+    if not torch.cuda.is_available():
+        assert chunk() in (-5, -6)                   # valid: stops at the device check
