@@ -24,7 +24,7 @@ namespace decode {
 
 constexpr int kThreads = 256;
 
-template <int DK, int DV, typename IO>
+template <int DK, int DV, typename IO, bool kRawGate>
 __global__ void __launch_bounds__(kThreads, 2) recurrent_step_kernel(StepArgs a) {
   constexpr int CG = DV / 4;         // column groups of 4 fp32
   constexpr int RG = kThreads / CG;  // row groups
@@ -34,6 +34,7 @@ __global__ void __launch_bounds__(kThreads, 2) recurrent_step_kernel(StepArgs a)
   __shared__ float red_k[RG][DV], red_q[RG][DV];
   __shared__ __align__(16) float delta[DV];
   __shared__ float kq_s;
+  __shared__ float gate_s[2];  // exp(g), beta
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int h = blockIdx.x, n = blockIdx.y;
@@ -45,14 +46,17 @@ __global__ void __launch_bounds__(kThreads, 2) recurrent_step_kernel(StepArgs a)
     for (int c = tid; c < DV; c += kThreads) static_cast<IO*>(a.out)[((size_t)n * a.nv + h) * DV + c] = from_f32<IO>(0.f);
     return;
   }
+  if (tid == 64) {  // warp 2 is idle while warps 0-1 normalise q and k; issued before the state loads
+    float gv, bv;
+    load_gate_t<kRawGate>(a, (size_t)n * a.nv + h, h, gv, bv);
+    gate_s[0] = expf(gv);
+    gate_s[1] = bv;
+  }
   float4* st = reinterpret_cast<float4*>(a.state + ((size_t)srow * a.nv + h) * (size_t)DK * DV);
   float4 s[RPT];
 #pragma unroll
   for (int i = 0; i < RPT; ++i) s[i] = __ldcs(st + (size_t)(i * RG + rg) * CG + cg);
 
-  float gv, bta;
-  load_gate(a, (size_t)n * a.nv + h, h, gv, bta);
-  const float alpha = expf(gv);
 
   // q_hat, k_hat (warp 0: q, warp 1: k)
   if (warp < 2) {
@@ -73,6 +77,7 @@ __global__ void __launch_bounds__(kThreads, 2) recurrent_step_kernel(StepArgs a)
     for (int e = 0; e < PER; ++e) dst[lane * PER + e] = x[e] * f;
   }
   __syncthreads();
+  const float alpha = gate_s[0], bta = gate_s[1];
   if (warp == 0) {
     float p = 0.f;
     for (int d = lane; d < DK; d += 32) p += qh[d] * kh[d];
@@ -126,7 +131,10 @@ __global__ void __launch_bounds__(kThreads, 2) recurrent_step_kernel(StepArgs a)
 template <int DK, int DV, typename IO>
 static cudaError_t launch_one(const StepArgs& a, cudaStream_t stream) {
   dim3 grid(a.nv, a.num_seqs);
-  recurrent_step_kernel<DK, DV, IO><<<grid, kThreads, 0, stream>>>(a);
+  if (a.A_log)
+    recurrent_step_kernel<DK, DV, IO, true><<<grid, kThreads, 0, stream>>>(a);
+  else
+    recurrent_step_kernel<DK, DV, IO, false><<<grid, kThreads, 0, stream>>>(a);
   return cudaGetLastError();
 }
 
