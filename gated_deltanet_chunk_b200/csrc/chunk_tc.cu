@@ -15,9 +15,9 @@
 //   serial warps (8-11): the state recurrence for this CTA's Dv slice.  The
 //     fp32 state slice S [128 x 64] lives in TMEM (lane d holds row d) and,
 //     rounded to bf16, in shared memory as the B operand of the next
-//     chunk.  The critical path per chunk is two tensor-core round trips
-//     (V', then D4) and two short epilogues; -W is formed before S is needed,
-//     and the output rows (P V' + Q S) are finished by warps 10-11 while
+//     chunk.  The critical path per chunk is three tensor-core round trips
+//     ([K;Q] S with U, then V', then D4) and three short epilogues; W itself
+//     is never formed.  The output rows (P V' + Q S) are finished by warps 10-11 while
 //     warps 8-9 start the next chunk.  The serial warps also refill this CTA's
 //     3-deep TMA ring of raw q/k/v tiles.
 //
@@ -32,9 +32,9 @@
 //   T  = (I - A)^-1 over 32 x 32 blocks, fp32 in shared memory:     CUDA cores
 //        T11, T22 by forward substitution on T = I + A T (one column per lane),
 //        T21 = T22 (A21 T11) (two 32 x 32 products over 256 threads)
-//   serial:  -W = (-T diag(beta exp(gcum) rk)) K                        one round
-//            V' = T diag(beta) V + (-W) S   (one accumulator)           one round
-//            [KS; QS] = [K; Q] S                                  same round, own use
+//   serial:  U = T diag(beta) V,  [K S; Q S] = [K; Q] S                one round
+//            K S rounded to bf16                                      CUDA cores
+//            V' = U + (-T diag(beta exp(gcum) rk)) (K S) = U - W S      one round
 //            D4 = K^T diag(rk exp(g_last - gcum)) V'                    one round
 //            PV = P V'                                            after D4, own use
 //            S <- exp(g_last) S + D4;  O = diag(exp(gcum) rq) QS + PV
@@ -106,7 +106,6 @@ static_assert(SMEM_BYTES <= 232448, "shared memory");
 constexpr uint32_t TM_G = 0;     // intra: G
 constexpr uint32_t TM_S = 64;    // serial: the fp32 state slice S (row d in lane d, 64 cols)
 constexpr uint32_t TM_QS = 192;  // serial: [K S ; Q S], two column blocks used alternately (128 cols)
-constexpr uint32_t TM_W = 320;   // serial: -W (128 cols: the U and D4 blocks, both free at that point)
 constexpr uint32_t TM_U = 320;   // serial: U - W S (rows 0..63)
 constexpr uint32_t TM_D4 = 384;  // serial: state update
 constexpr uint32_t TM_PV = 448;  // serial: P V' (rows 64..127)
@@ -591,7 +590,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float* spp = sp + psl * SP_N;
       const uint32_t tm_qs = TM_QS + 64u * par;  // [K S; Q S] alternates between two column blocks
       if (vrow) {
-        // -W = (-T diag(bw)) K   (A = [-T diag(bw); junk])
+        // U = T diag(beta) V and [K S; Q S]
         if (t == 0) {
           if (!ptx::mbar_wait_bounded(bars + BAR_RAWF + rsl, (uint32_t)((c / NR) & 1), kWaitNs) ||
               !ptx::mbar_wait_cluster_bounded(bars + BAR_PRODF + psl, (uint32_t)((c / NP) & 1), kWaitNs))
@@ -599,7 +598,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (*abort_flag == 0) {
             ptx::fence_proxy_async_smem();  // products stored by threads (possibly of the other CTA)
             ptx::tc_fence_after();
-            mma_k64(tmem + TM_W, pa + PS_WHI, ra + RS_KLO, RS_KHI - RS_KLO, ID_KMN128, 0);
+            mma_k64(tmem + TM_U, pa + PS_TU, ra + RS_V, 8192, ID_KMN64, 0);
+            mma_k128(tmem + tm_qs, ra + RS_KLO, ra + RS_KHI, sb + OFF_S, 8192, ID_KMN64, 0);
             ptx::mma_commit(bars + BAR_MMAW);
             if (!ptx::mbar_wait_bounded(bars + BAR_MMAW, par, kWaitNs)) *abort_flag = 1;
           }
@@ -608,25 +608,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = (*abort_flag == 0);
         ptx::tc_fence_after();
         if (ok) {
-#pragma unroll
-          for (int qq = 0; qq < 4; ++qq) {  // row t of -W, 32 columns at a time, into W_lo | W_hi
-            float x[32];
-            ptx::tmem_ld32(tl + TM_W + 32 * qq, x);
-            ptx::tmem_ld_wait();
-            ptx::st_half_bf16(ps + (qq < 2 ? PS_WLO : PS_WHI), t, qq & 1, x);
-          }
+          // row t of K S, rounded to bf16, into W_lo: the B operand of the next product
+          float x[64];
+          tmem_row64(tl + tm_qs, x);
+          ptx::st_row_bf16(ps + PS_WLO, t, x);
         }
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
         named_bar_n(3, 64);
-        // U - W S and [K S; Q S]
+        // V' = U + (-T diag(bw)) (K S) = U - W S   (A = [-T diag(bw); junk])
         if (t == 0) {
           if (*abort_flag == 0) {
             ptx::tc_fence_after();
-            mma_k64(tmem + TM_U, pa + PS_TU, ra + RS_V, 8192, ID_KMN64, 0);
-            mma_k128(tmem + TM_U, pa + PS_WLO, pa + PS_WHI, sb + OFF_S, 8192, ID_KMN64, 1);
+            mma_k64(tmem + TM_U, pa + PS_WHI, pa + PS_WLO, 8192, ID_KMN64, 1);
             ptx::mma_commit(bars + BAR_MMAS);
-            mma_k128(tmem + tm_qs, ra + RS_KLO, ra + RS_KHI, sb + OFF_S, 8192, ID_KMN64, 0);
             if (!ptx::mbar_wait_bounded(bars + BAR_MMAS, par, kWaitNs)) *abort_flag = 1;
           }
         }
