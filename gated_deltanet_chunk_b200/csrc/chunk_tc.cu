@@ -113,7 +113,6 @@ constexpr uint32_t TM_COLS = 512;
 
 constexpr uint32_t ID_KK64 = ptx::idesc_bf16_f32(128, 64, false, false);
 constexpr uint32_t ID_KMN64 = ptx::idesc_bf16_f32(128, 64, false, true);
-constexpr uint32_t ID_KMN128 = ptx::idesc_bf16_f32(128, 128, false, true);
 constexpr uint32_t ID_MNMN64 = ptx::idesc_bf16_f32(128, 64, true, true);
 
 // exp(x) as 2^(x log2 e) on the special-function unit, flushing results below
