@@ -96,7 +96,7 @@ constexpr int OFF_BAR = OFF_SCP + NP * SP_N * 4;
 // peer_free[NP] (the other CTA's serial warps are done with its copy); mma_i, mma_s
 constexpr int BAR_RAWF = 0, BAR_PRODF = NR, BAR_PRODE = NR + NP, BAR_PEERF = NR + 2 * NP;
 constexpr int BAR_MMAI = NR + 3 * NP, BAR_MMAS = BAR_MMAI + 1, BAR_MMAD4 = BAR_MMAS + 1, BAR_MMAO = BAR_MMAD4 + 1;
-constexpr int BAR_OUTD = BAR_MMAO + 1, BAR_MMAW = BAR_OUTD + 1, NBAR = BAR_MMAW + 1;
+constexpr int BAR_OUTD = BAR_MMAO + 1, BAR_MMAW = BAR_OUTD + 1, BAR_DRAIN = BAR_MMAW + 1, NBAR = BAR_DRAIN + 1;
 constexpr int SMEM_USED = OFF_BAR + NBAR * 8 + 16;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
 static_assert(OFF_BAR % 8 == 0, "mbarrier alignment");
@@ -204,6 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::mbar_init(bars + BAR_MMAO, 1);
     ptx::mbar_init(bars + BAR_OUTD, 2);
     ptx::mbar_init(bars + BAR_MMAW, 1);
+    ptx::mbar_init(bars + BAR_DRAIN, 3);  // one commit per MMA-issuing thread
     *abort_flag = 0;
     ptx::fence_mbar_init();
     ptx::prefetch_tensormap(&tm_q);
@@ -653,6 +654,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mma_bf16(tmem + TM_D4, mndesc(ra + RS_KLO + 2048 * kk, RS_KHI - RS_KLO),
                           mndesc(pa + PS_WHI + 2048 * kk, 8192), ID_MNMN64, kk > 0);
           ptx::mma_commit(bars + BAR_MMAD4);
+        }
+        if (t == 32 && *abort_flag == 0) {  // off the polling thread's path
+          ptx::tc_fence_after();
           if (c > 0 && !ptx::mbar_wait_bounded(bars + BAR_OUTD, par ^ 1u, kWaitNs)) *abort_flag = 1;
           ptx::tc_fence_after();
           mma_k64(tmem + TM_PV, pa + PS_P - kTile, pa + PS_WLO, 8192, ID_KMN64, 0);
@@ -755,10 +759,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!ok && t == 0) atomicOr(&g_status, 1u);
   }
 
+  // Every thread that issued MMAs (intra 0, serial 0 and 32) commits once more:
+  // on an early exit some of its MMAs may still be running, and TMEM is freed
+  // only after they have completed (bounded, like every wait here).
+  if (tid == 0 || tid == 256 || tid == 288) ptx::mma_commit(bars + BAR_DRAIN);
   ptx::tc_fence_before();
   __syncthreads();
   ptx::cluster_sync_all();  // the other CTA no longer touches this CTA's shared memory
   if (warp == 0) {
+    if (lane == 0 && !ptx::mbar_wait_bounded(bars + BAR_DRAIN, 0u, kWaitNs)) atomicOr(&g_status, 1u);
+    __syncwarp();
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, TM_COLS);
   }
