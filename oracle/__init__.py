@@ -19,6 +19,11 @@ This module only marshals arrays:
 * :func:`chunk_prepare` -- the intra-chunk quantities of one chunk (gate
   cumsum, decay mask, A, T = (I - A)^-1, U, W), for the inverse and similarity
   pins.
+* :func:`gated_rmsnorm` -- the output epilogue (RMSNormGated, walkthrough
+  sections 1 and 6): y = o / sqrt(mean(o^2) + eps) * w * silu(z).
+* :func:`causal_conv1d` -- the causal depthwise conv1d + SiLU of the packed
+  q|k|v channels with its conv_state window (walkthrough section 3; prefill and
+  torch_causal_conv1d_update).
 
 Inputs may be numpy arrays or CPU torch tensors of any float dtype (bf16
 included); they are upcast exactly to fp64.  Outputs are fp64 numpy arrays.
@@ -71,6 +76,10 @@ def _load():
         lib.oracle_chunk_prepare.argtypes = [i, i, i, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp]
         lib.oracle_gates.argtypes = [ctypes.c_int64, i, dp, dp, dp, dp, dp, dp]
         lib.oracle_chunk_prepare.restype = i
+        lib.oracle_gated_rmsnorm.argtypes = [ctypes.c_int64, i, dp, dp, dp, ctypes.c_double, dp]
+        lib.oracle_gated_rmsnorm.restype = i
+        lib.oracle_causal_conv1d.argtypes = [i, ip, i, i, dp, dp, dp, dp, dp, dp]
+        lib.oracle_causal_conv1d.restype = i
         _lib = lib
     return _lib
 
@@ -191,3 +200,47 @@ def gates(a, b, A_log, dt_bias):
     if rc != 0:
         raise ValueError("oracle_gates failed (%d)" % rc)
     return g, beta
+
+
+def gated_rmsnorm(o, z, weight, eps=1e-6):
+    """y = o / sqrt(mean(o^2) + eps) * weight * silu(z) over the last axis (oracle_gated_rmsnorm).
+
+    ``o`` and ``z`` have the same shape [..., Dv]; ``weight`` is [Dv].  Returns a
+    float64 numpy array of that shape.
+    """
+    o64, z64, w64 = _f64(o), _f64(z), _f64(weight).reshape(-1)
+    dv = o64.shape[-1]
+    if z64.shape != o64.shape or w64.shape[0] != dv:
+        raise ValueError("gated_rmsnorm: o, z [..., Dv] and weight [Dv] expected")
+    y = np.empty_like(o64)
+    rc = _load().oracle_gated_rmsnorm(o64.size // dv, dv, _ptr(o64), _ptr(z64), _ptr(w64),
+                                      float(eps), _ptr(y))
+    if rc != 0:
+        raise ValueError("oracle_gated_rmsnorm: bad arguments (%d)" % rc)
+    return y
+
+
+def causal_conv1d(x, weight, bias=None, cu_seqlens=None, conv_state=None):
+    """Causal depthwise conv1d + SiLU per sequence (oracle_causal_conv1d).
+
+    ``x`` is [T, channels] (token-major), ``weight`` [channels, ksize], ``bias``
+    [channels] or None, ``conv_state`` [N, channels, ksize] or None (zeros): the
+    ksize inputs before each sequence.  Returns ``(y [T, channels],
+    new_conv_state [N, channels, ksize])`` as float64 numpy arrays.
+    """
+    x64, w64 = _f64(x), _f64(weight)
+    T, ch = x64.shape
+    ks = w64.shape[1]
+    if w64.shape[0] != ch:
+        raise ValueError("causal_conv1d: weight [channels, ksize] expected")
+    cu = _i32(np.array([0, T]) if cu_seqlens is None else cu_seqlens)
+    n = len(cu) - 1
+    b64 = _f64(bias)
+    s64 = _f64(conv_state)
+    y = np.empty_like(x64)
+    s_out = np.zeros((n, ch, ks))
+    rc = _load().oracle_causal_conv1d(n, _ptr(cu), ch, ks, _ptr(x64), _ptr(w64), _ptr(b64),
+                                      _ptr(s64), _ptr(y), _ptr(s_out))
+    if rc != 0:
+        raise ValueError("oracle_causal_conv1d: bad arguments (%d)" % rc)
+    return y, s_out

@@ -21,6 +21,14 @@
  *   oracle_gates       -- beta = sigmoid(b);  g = -exp(A_log) * softplus(a + dt_bias)
  *                         with softplus(x) = log(1 + exp(x)), per token and v-head.
  *
+ * The layer steps around it, on the same page (NEXT to the core, same rules):
+ *
+ *   oracle_gated_rmsnorm -- output epilogue, [WT] 一(一)1 and 6: RMSNormGated,
+ *                         y = o / sqrt(mean(o^2) + eps) * w * silu(z).
+ *   oracle_causal_conv1d -- [WT] 一(一)3: causal depthwise conv1d + SiLU of the
+ *                         packed q|k|v channels, with the conv_state window of
+ *                         torch_causal_conv1d_update (prefill and decode).
+ *
  * Two functions compute the method:
  *
  *   oracle_recurrent   -- THE DEFINITION.  Token loop of [WT] (2):
@@ -342,6 +350,88 @@ int oracle_gates(int64_t T, int nv, const double *a, const double *b, const doub
             g[i] = -exp(A_log[h]) * sp;
             beta[i] = 1.0 / (1.0 + exp(-b[i]));
         }
+    }
+    return 0;
+}
+
+/* ---------------------------------------------------------------------------
+ * Output epilogue: gated RMSNorm (RMSNormGated), per row of head_v_dim values.
+ *
+ * [WT] section 一(一)1 builds the layer's norm as RMSNormGated(head_v_dim,
+ * eps) and section 一(一)6 (输出调整) applies it as norm(o, z) with o and z
+ * flattened to rows of head_v_dim: "RMSNorm + Gate".  The page says this
+ * norm is the ordinary RMSNorm with a gain initialised to 1; its RMSNorm code
+ * (section 三, Zero-Centered RMSNorm, _norm) multiplies x by
+ * rsqrt(mean(x^2) + eps).  The gate's activation is not printed: it is read
+ * as SiLU, z * sigmoid(z), applied to z after the norm:
+ *
+ *     y = o / sqrt(mean(o^2) + eps) * w * silu(z),   silu(x) = x / (1 + exp(-x))
+ *
+ * o, z, y are [rows, dv]; w is [dv].
+ * ------------------------------------------------------------------------- */
+int oracle_gated_rmsnorm(int64_t rows, int dv, const double *o, const double *z,
+                         const double *w, double eps, double *y)
+{
+    if (rows < 0 || dv <= 0 || !o || !z || !w || !y || !(eps >= 0.0)) return -1;
+    for (int64_t r = 0; r < rows; ++r) {
+        const double *orow = o + r * dv, *zrow = z + r * dv;
+        double ms = 0.0;
+        for (int c = 0; c < dv; ++c) ms += orow[c] * orow[c];
+        ms /= (double)dv;
+        const double inv = 1.0 / sqrt(ms + eps);
+        for (int c = 0; c < dv; ++c) {
+            const double gate = zrow[c] / (1.0 + exp(-zrow[c]));
+            y[r * dv + c] = orow[c] * inv * w[c] * gate;
+        }
+    }
+    return 0;
+}
+
+/* ---------------------------------------------------------------------------
+ * Causal depthwise conv1d + SiLU over the packed q|k|v channels.
+ *
+ * [WT] section 一(一)3 (qkv 卷积部分): every channel is convolved on its own
+ * (groups = channels) with a kernel of `ksize` taps, zero padded by ksize - 1
+ * on the left and cut to the sequence length, then passed through SiLU.  Tap i
+ * of channel c multiplies input t - (ksize - 1) + i (cross-correlation, as
+ * torch's conv1d computes it), so tap ksize - 1 meets the current token.  The
+ * decode update (torch_causal_conv1d_update) is the same computation over
+ * [conv_state, x]: the window before a sequence is the cached conv_state of
+ * ksize pre-convolution inputs (zeros for a fresh prefill), and the new
+ * conv_state is the last ksize inputs of [window, sequence], zero filled on
+ * the left when fewer exist.
+ *
+ *   x, y       [T, channels] (token-major)  sequence n owns tokens [cu[n], cu[n+1])
+ *   w          [channels, ksize]            bias [channels] or NULL
+ *   state_in   [N, channels, ksize] or NULL (zeros); state_out likewise or NULL.
+ *              state_out may be state_in (updated in place).
+ * ------------------------------------------------------------------------- */
+int oracle_causal_conv1d(int num_seqs, const int32_t *cu, int channels, int ksize,
+                         const double *x, const double *w, const double *bias,
+                         const double *state_in, double *y, double *state_out)
+{
+    if (num_seqs < 1 || !cu || channels <= 0 || ksize < 1 || !x || !w || !y) return -1;
+    if (cu[0] != 0) return -2;
+    for (int n = 0; n < num_seqs; ++n)
+        if (cu[n + 1] < cu[n]) return -2;
+#pragma omp parallel for schedule(dynamic, 16)
+    for (long p = 0; p < (long)num_seqs * channels; ++p) {
+        const int n = (int)(p / channels), c = (int)(p % channels);
+        const int64_t t0 = cu[n], len = (int64_t)cu[n + 1] - cu[n];
+        const size_t sidx = ((size_t)n * channels + c) * ksize;
+        /* extended input: the ksize-entry window, then the sequence */
+        double *ext = (double *)malloc(sizeof(double) * (size_t)(ksize + len));
+        for (int i = 0; i < ksize; ++i) ext[i] = state_in ? state_in[sidx + i] : 0.0;
+        for (int64_t t = 0; t < len; ++t) ext[ksize + t] = x[(t0 + t) * channels + c];
+        for (int64_t t = 0; t < len; ++t) {
+            /* token t sits at ext[ksize + t]; tap i reads ext[ksize + t - (ksize-1) + i] */
+            double pre = bias ? bias[c] : 0.0;
+            for (int i = 0; i < ksize; ++i) pre += w[(size_t)c * ksize + i] * ext[t + 1 + i];
+            y[(t0 + t) * channels + c] = pre / (1.0 + exp(-pre));
+        }
+        if (state_out)
+            for (int i = 0; i < ksize; ++i) state_out[sidx + i] = ext[len + i];
+        free(ext);
     }
     return 0;
 }

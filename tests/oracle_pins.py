@@ -352,6 +352,115 @@ def pin_gates_closed_forms():
     assert abs(gt[0, 1] / -A[1] / np.exp(-40.0) - 1.0) < 1e-12
 
 
+def pin_gated_rmsnorm():
+    """Output epilogue (walkthrough sections 1 and 6, RMSNormGated; its RMSNorm
+    code in section 3): y = o / sqrt(mean(o^2) + eps) * w * silu(z).
+
+    Pinned by what the definitions fix, not by retyping them:
+    - with eps = 0 the normalised part has unit mean square over Dv;
+    - eps sits inside the root: for a constant row o = c the ratio
+      y / (w silu(z)) is 1 / sqrt(1 + eps / c^2) (eps outside would give c / (|c| + eps));
+    - homogeneity: y(a o, a^2 eps) = y(o, eps) for a > 0, and y is linear in w;
+    - the gate is SiLU of z: silu(0) = 0; silu(x) - silu(-x) = x; and
+      silu(x) / silu(-x) = -exp(x), which fixes the logistic factor (x * Phi(x)
+      would give -Phi(x) / Phi(-x));
+    - rows are independent: permuting rows permutes y.
+    """
+    rng = np.random.default_rng(21)
+    R, dv = 9, 16
+    o = rng.standard_normal((R, dv)) * rng.uniform(0.1, 5.0, size=(R, 1))
+    z = rng.standard_normal((R, dv)) * 3.0
+    w = rng.uniform(0.5, 2.0, size=dv)
+    y0 = oracle.gated_rmsnorm(o, z, w, eps=0.0)
+    gate = oracle.gated_rmsnorm(np.ones((R, dv)), z, w, eps=0.0) / w  # = silu(z): o = 1 has rms 1
+    n = y0 / (w * gate)
+    assert np.max(np.abs(np.mean(n * n, axis=1) - 1.0)) < 1e-12
+    # eps placement on constant rows
+    for c_, eps in ((1e-3, 1e-6), (2.0, 0.5), (-0.3, 1e-2)):
+        yc = oracle.gated_rmsnorm(np.full((1, dv), c_), np.full((1, dv), 2.0), np.ones(dv), eps)
+        yg = oracle.gated_rmsnorm(np.ones((1, dv)), np.full((1, dv), 2.0), np.ones(dv), 0.0)
+        ratio = yc / yg
+        assert np.max(np.abs(ratio - np.sign(c_) / np.sqrt(1.0 + eps / c_ ** 2))) < 1e-13
+    # homogeneity and linearity in w
+    a = 7.5
+    y1 = oracle.gated_rmsnorm(o, z, w, eps=1e-3)
+    assert rel(oracle.gated_rmsnorm(a * o, z, w, eps=a * a * 1e-3), y1) < 1e-13
+    assert rel(oracle.gated_rmsnorm(o, z, 3.0 * w, eps=1e-3), 3.0 * y1) < 1e-14
+    # SiLU of z
+    assert np.all(oracle.gated_rmsnorm(o, np.zeros_like(z), w, 1e-3) == 0.0)
+    zz = np.linspace(-20.0, 20.0, dv)[None, :].repeat(R, axis=0)
+    zz[:, dv // 2] = 0.7  # keep clear of x = 0
+    yp = oracle.gated_rmsnorm(o, zz, w, 1e-3)
+    ym = oracle.gated_rmsnorm(o, -zz, w, 1e-3)
+    base = oracle.gated_rmsnorm(o, np.ones_like(zz), w, 1e-3) / \
+        oracle.gated_rmsnorm(np.ones((R, dv)), np.ones_like(zz), np.ones(dv), 0.0)  # o/rms * w
+    assert rel((yp - ym) / base, zz) < 1e-12
+    assert np.max(np.abs(yp / ym / -np.exp(zz) - 1.0)) < 1e-12
+    perm = rng.permutation(R)
+    assert np.array_equal(oracle.gated_rmsnorm(o[perm], z[perm], w, 1e-3), y1[perm])
+
+
+def _conv_ref_pre(x, w, bias, window):
+    """Pre-activation of one channel by numpy's full convolution of [window, x]
+    with the reversed taps (a cross-correlation), cut to the sequence."""
+    ks = len(w)
+    ext = np.concatenate([window, x])
+    full = np.convolve(ext, w[::-1])  # full[m] = sum_i w[i] ext[m - (ks-1) + i]
+    return full[ks: ks + len(x)] + bias
+
+
+def pin_causal_conv1d():
+    """Causal depthwise conv1d + SiLU (walkthrough section 3) and its conv_state.
+
+    Pinned by numpy's own convolution (np.convolve with reversed taps, i.e. the
+    cross-correlation of torch's conv1d) for the pre-activation, and by the
+    logistic identities of SiLU: y(x) - y(-x) = pre and y(x) / y(-x) = -exp(pre)
+    (inputs, bias and window negated together negate pre).  The state rules:
+    the new conv_state is the last ksize inputs of [window, sequence]; one run
+    equals the same tokens split in two with the state carried across, and
+    equals one decode step per token (torch_causal_conv1d_update); channels and
+    sequences are independent.
+    """
+    rng = np.random.default_rng(22)
+    ch, ks = 5, 4
+    lens = [1, 3, 4, 9, 17]
+    T = sum(lens)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    x = rng.standard_normal((T, ch))
+    w = rng.standard_normal((ch, ks))
+    bias = rng.standard_normal(ch)
+    st = rng.standard_normal((len(lens), ch, ks))
+    for window in (None, st):
+        yp, sp = oracle.causal_conv1d(x, w, bias, cu, window)
+        ym, _ = oracle.causal_conv1d(-x, w, -bias, cu, None if window is None else -window)
+        for n, L in enumerate(lens):
+            for c in range(ch):
+                win = np.zeros(ks) if window is None else window[n, c]
+                pre = _conv_ref_pre(x[cu[n]:cu[n + 1], c], w[c], bias[c], win)
+                seg_p, seg_m = yp[cu[n]:cu[n + 1], c], ym[cu[n]:cu[n + 1], c]
+                assert np.max(np.abs((seg_p - seg_m) - pre)) < 1e-12
+                ok = np.abs(pre) > 1e-3
+                assert np.max(np.abs(seg_p[ok] / seg_m[ok] / -np.exp(pre[ok]) - 1.0)) < 1e-11
+                ext = np.concatenate([win, x[cu[n]:cu[n + 1], c]])
+                assert np.array_equal(sp[n, c], ext[-ks:])
+    # split with the state carried = one run; per-token decode = one run
+    x1 = rng.standard_normal((23, ch))
+    y_all, s_all = oracle.causal_conv1d(x1, w, bias, None, st[:1])
+    ya, sa = oracle.causal_conv1d(x1[:10], w, bias, None, st[:1])
+    yb, sb = oracle.causal_conv1d(x1[10:], w, bias, None, sa)
+    assert rel(np.concatenate([ya, yb]), y_all) < 1e-15 and np.array_equal(sb, s_all)
+    s_dec = st[:1].copy()
+    for t in range(23):
+        yt, s_dec = oracle.causal_conv1d(x1[t:t + 1], w, bias, None, s_dec)
+        assert rel(yt, y_all[t:t + 1]) < 1e-15
+    assert np.array_equal(s_dec, s_all)
+    # causality: changing a later token leaves earlier outputs unchanged
+    x2 = x1.copy()
+    x2[15] += 1.0
+    y2, _ = oracle.causal_conv1d(x2, w, bias, None, st[:1])
+    assert np.array_equal(y2[:15], y_all[:15]) and not np.array_equal(y2[15], y_all[15])
+
+
 # --------------------------------------------------------------------------
 # Stored golden values (tests/golden/*.txt): outputs of small cases written by
 # tests/golden/make_golden.py from the oracle, so a later change of the oracle's
@@ -363,4 +472,5 @@ ALL_PINS = [
     pin_chunk_equals_recurrent, pin_beta_zero, pin_delta_write_exact, pin_zero_pad_invariance,
     pin_split_carry_and_varlen, pin_gqa_repeat_interleave, pin_linearity, pin_orthonormal_keys,
     pin_dv_columns_independent, pin_inverse_and_similarity, pin_gates_closed_forms,
+    pin_gated_rmsnorm, pin_causal_conv1d,
 ]

@@ -59,6 +59,25 @@ MUTANTS = [
     ("key_decay_wrong", "exp(glast - gc[i])", "exp(gc[i])", 0),
     ("inter_no_decay", "s1 += Qc[(size_t)r * dk + d] * eg * S[(size_t)d * dv + x];",
      "s1 += Qc[(size_t)r * dk + d] * S[(size_t)d * dv + x];", 0),
+    # gated RMSNorm epilogue
+    ("norm_eps_outside_root", "const double inv = 1.0 / sqrt(ms + eps);",
+     "const double inv = 1.0 / (sqrt(ms) + eps);", 0),
+    ("norm_sum_not_mean", "ms /= (double)dv;", "ms /= 1.0;", 0),
+    ("norm_gate_sigmoid", "const double gate = zrow[c] / (1.0 + exp(-zrow[c]));",
+     "const double gate = 1.0 / (1.0 + exp(-zrow[c]));", 0),
+    ("norm_gate_on_o", "const double gate = zrow[c] / (1.0 + exp(-zrow[c]));",
+     "const double gate = zrow[c] / (1.0 + exp(-orow[c]));", 0),
+    # causal conv1d + SiLU
+    ("conv_taps_shifted", "pre += w[(size_t)c * ksize + i] * ext[t + 1 + i];",
+     "pre += w[(size_t)c * ksize + i] * ext[t + i];", 0),
+    ("conv_taps_reversed", "pre += w[(size_t)c * ksize + i] * ext[t + 1 + i];",
+     "pre += w[(size_t)c * ksize + (ksize - 1 - i)] * ext[t + 1 + i];", 0),
+    ("conv_no_silu", "y[(t0 + t) * channels + c] = pre / (1.0 + exp(-pre));",
+     "y[(t0 + t) * channels + c] = pre;", 0),
+    ("conv_state_ignored", "ext[i] = state_in ? state_in[sidx + i] : 0.0;", "ext[i] = 0.0;", 0),
+    ("conv_no_bias", "double pre = bias ? bias[c] : 0.0;", "double pre = 0.0;", 0),
+    ("conv_state_not_advanced", "state_out[sidx + i] = ext[len + i];",
+     "state_out[sidx + i] = ext[i];", 0),
 ]
 
 CHILD = r"""
