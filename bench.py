@@ -192,6 +192,32 @@ def time_oracle(w, T_sample, heads=None):
 
 
 # --------------------------------------------------------------------------- main
+def time_steps(fn, warmup, steps, stream, world, dev):
+    """Device time per call of ``fn`` (CUDA events on ``stream``, max over ranks), after warm-up."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    return max_over_ranks(a.elapsed_time(b), world, dev) / steps
+
+
+def hbm_line(ms, byts, peaks, peak_src, **extra):
+    gbs = byts / (ms / 1e3) / 1e9
+    r = {"ms_per_step": ms, "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                                         "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                                         "peak_source": peak_src, "alg_bytes_per_launch": byts}}
+    r.update(extra)
+    return r
+
+
 def run_ours(args, world, rank, local):
     import torch
 
@@ -296,6 +322,28 @@ def run_ours(args, world, rank, local):
                                      "traffic": None, "peak_source": peak_src,
                                      "alg_bytes_per_launch": g_bytes}}
         del ga
+    # the same workload with the gated RMSNorm epilogue fused into the output
+    # stores (gdn_chunk_fwd_ex), and the epilogue on its own (gdn_gated_rmsnorm)
+    if not args.no_norm:
+        z, nw = W.make_norm_inputs((T, nv, D), "bf16", seed=2 + rank, device=str(dev))
+
+        def nstep():
+            gdn.chunk_fwd_ex(d["q"], d["k"], d["v"], d["g"], d["beta"], None, None, chunk_size=C, out=out,
+                             final_state=sf, num_seqs=n, norm_z=z, norm_weight=nw, norm_eps=1e-6)
+
+        n_ms = time_steps(nstep, args.warmup, args.steps, stream, world, dev)
+        zb = T * nv * D * 2 + D * 4
+        res["normed"] = hbm_line(n_ms, bytes_alg + zb, peaks, peak_src, value=T * world / (n_ms / 1e3),
+                                 unit="tokens/s", call="gdn_chunk_fwd_ex (norm_z): chunk kernel + norm pass",
+                                 gpu_launches=2 * args.steps)
+        y = torch.empty_like(out)
+        r_ms = time_steps(lambda: gdn.gated_rmsnorm(out, z, nw, 1e-6, out=y), args.warmup, args.steps,
+                          stream, world, dev)
+        res["gated_rmsnorm"] = hbm_line(r_ms, 3 * T * nv * D * 2 + D * 4, peaks, peak_src,
+                                        value=T * world / (r_ms / 1e3), unit="tokens/s",
+                                        call="gdn_gated_rmsnorm", rows=T * nv, dim=D,
+                                        gpu_launches=args.steps)
+        del z, y
     # e2e: same call with host buffers (pinned), copies inside the timed region
     if not args.no_e2e:
         hp = {k: host[k].pin_memory() for k in ("q", "k", "v", "g", "beta")}
@@ -428,6 +476,21 @@ def run_decode(args, world, rank, dev, stream, peaks, peak_src):
                                      "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                      "frac": gb / (gms / 1e3) / 1e9 / peaks["hbm_gbs"], "traffic": None,
                                      "peak_source": peak_src, "alg_bytes_per_launch": gb}}
+    if not args.no_norm:
+        z, nw = W.make_norm_inputs((steps, wl.num_seqs, wl.nv, wl.d), "bf16", seed=4 + rank, device=str(dev))
+        it = [0]
+
+        def run_normed():
+            t = it[0] % steps
+            it[0] += 1
+            gdn.recurrent_step_ex(d["q"][t], d["k"][t], d["v"][t], d["g"][t], d["beta"][t], state, out=out,
+                                  norm_z=z[t], norm_weight=nw, norm_eps=1e-6)
+
+        nms = time_steps(run_normed, min(steps, 32), steps, stream, world, dev)
+        nb = byts + wl.num_seqs * wl.nv * wl.d * 2 + wl.d * 4
+        res["normed"] = hbm_line(nms, nb, peaks, peak_src, value=wl.num_seqs * world / (nms / 1e3),
+                                 unit="tokens/s", call="gdn_recurrent_step_ex (norm_z)", gpu_launches=steps)
+        del z
     return res
 
 
@@ -478,6 +541,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-gated", action="store_true", help="skip the fused-gate prefill and decode lines")
     ap.add_argument("--no-slots", action="store_true", help="skip the slot-indexed decode line")
+    ap.add_argument("--no-norm", action="store_true",
+                    help="skip the gated-RMSNorm lines (fused prefill and decode, standalone epilogue)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=0,
                     help="oracle sample per sequence for cpu_baseline (default: the whole workload)")

@@ -10,6 +10,11 @@ Functions
 ---------
 chunk_fwd(q, k, v, g, beta, ...)       -> (out, final_state)   prefill, gdn_chunk_fwd
 recurrent_step(q, k, v, g, beta, state, ...) -> out            decode, gdn_recurrent_step
+chunk_fwd_gated / recurrent_step_gated                         the gate formed in-kernel
+chunk_fwd_slots / recurrent_step_slots                         states in a slot-indexed pool
+chunk_fwd_ex / recurrent_step_ex                               any of those fusions plus the
+                                                               gated RMSNorm epilogue (gdn_ext_t)
+gated_rmsnorm(o, z, weight, eps)       -> y                    the epilogue alone, gdn_gated_rmsnorm
 """
 from __future__ import annotations
 
@@ -38,6 +43,12 @@ class GdnParams(ctypes.Structure):
                 ("head_k_dim", ctypes.c_int32), ("head_v_dim", ctypes.c_int32),
                 ("io_dtype", ctypes.c_int32), ("qk_l2norm", ctypes.c_int32),
                 ("scale", ctypes.c_float), ("kernel", ctypes.c_int32)]
+
+
+class GdnExt(ctypes.Structure):
+    _fields_ = [("A_log", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p), ("slot_ids", ctypes.c_void_p),
+                ("num_slots", ctypes.c_int32), ("norm_z", ctypes.c_void_p), ("norm_weight", ctypes.c_void_p),
+                ("norm_eps", ctypes.c_float)]
 
 
 _lib = None
@@ -72,6 +83,16 @@ def lib() -> ctypes.CDLL:
         L.gdn_recurrent_step_slots.argtypes = [vp, vp, vp, fp, fp, fp, ip, ctypes.c_int32, vp, ctypes.c_int32,
                                                ctypes.POINTER(GdnParams), vp]
         L.gdn_recurrent_step_slots.restype = ctypes.c_int
+        L.gdn_chunk_fwd_ex.argtypes = [vp, vp, vp, fp, fp, fp, ip, ctypes.c_int32, ctypes.c_int64,
+                                       ctypes.c_int32, vp, fp, ctypes.POINTER(GdnParams),
+                                       ctypes.POINTER(GdnExt), vp]
+        L.gdn_chunk_fwd_ex.restype = ctypes.c_int
+        L.gdn_recurrent_step_ex.argtypes = [vp, vp, vp, fp, fp, fp, vp, ctypes.c_int32,
+                                            ctypes.POINTER(GdnParams), ctypes.POINTER(GdnExt), vp]
+        L.gdn_recurrent_step_ex.restype = ctypes.c_int
+        L.gdn_gated_rmsnorm.argtypes = [vp, vp, fp, ctypes.c_float, vp, ctypes.c_int64, ctypes.c_int32,
+                                        ctypes.c_int32, vp]
+        L.gdn_gated_rmsnorm.restype = ctypes.c_int
         L.gdn_device_status.argtypes = [vp]
         L.gdn_device_status.restype = ctypes.c_int
         L.gdn_status_string.argtypes = [ctypes.c_int]
@@ -221,4 +242,84 @@ def recurrent_step_slots(q, k, v, g, beta, state_pool, slot_ids, out=None, qk_l2
                                         ctypes.byref(p), _stream(stream))
     if check and rc != GDN_OK:
         raise GdnError(rc, "gdn_recurrent_step_slots")
+    return out
+
+
+def make_ext(A_log=None, dt_bias=None, slot_ids=None, num_slots=0, norm_z=None, norm_weight=None,
+             norm_eps=1e-6) -> GdnExt:
+    """The gdn_ext_t block: fused gate, slot pool and gated RMSNorm epilogue (each optional)."""
+    p = lambda t: None if t is None else t.data_ptr()
+    return GdnExt(p(A_log), p(dt_bias), p(slot_ids), int(num_slots), p(norm_z), p(norm_weight),
+                  float(norm_eps))
+
+
+def chunk_fwd_ex(q, k, v, g, beta, initial_state=None, cu_seqlens=None, chunk_size=64, out=None,
+                 final_state=None, output_final_state=True, num_seqs=None, qk_l2norm=True, scale=0.0,
+                 kernel="auto", A_log=None, dt_bias=None, slot_ids=None, norm_z=None, norm_weight=None,
+                 norm_eps=1e-6, stream=None, check=True):
+    """``chunk_fwd`` with any of the fusions of ``gdn_chunk_fwd_ex``.
+
+    A_log, dt_bias: the g, beta arguments are the raw projections a, b.
+    slot_ids: ``initial_state`` is a state pool [P, Nv, Dk, Dv], updated in place.
+    norm_z [T, Nv, Dv] (dtype of v), norm_weight [Dv] fp32: out holds
+    o / sqrt(mean(o^2) + norm_eps) * norm_weight * silu(norm_z) per row.
+    Returns ``(out, final_state)``.
+    """
+    import torch
+    T, nqk, dk = q.shape
+    nv, dv = v.shape[1], v.shape[2]
+    if slot_ids is not None:
+        n = slot_ids.numel()
+        final_state = initial_state
+    else:
+        n = (cu_seqlens.numel() - 1) if cu_seqlens is not None else (num_seqs or 1)
+        if final_state is None and output_final_state:
+            final_state = torch.empty((n, nv, dk, dv), dtype=torch.float32, device=v.device)
+    if out is None:
+        out = torch.empty((T, nv, dv), dtype=v.dtype, device=v.device)
+    p = make_params(nqk, nv, dk, dv, q.dtype == torch.bfloat16, qk_l2norm, scale, kernel)
+    x = make_ext(A_log, dt_bias, slot_ids, 0 if initial_state is None or slot_ids is None
+                 else initial_state.shape[0], norm_z, norm_weight, norm_eps)
+    rc = lib().gdn_chunk_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state),
+                                _ptr(cu_seqlens), int(n), int(T), int(chunk_size), _ptr(out),
+                                _ptr(final_state), ctypes.byref(p), ctypes.byref(x), _stream(stream))
+    if check and rc != GDN_OK:
+        raise GdnError(rc, "gdn_chunk_fwd_ex")
+    return out, final_state
+
+
+def recurrent_step_ex(q, k, v, g, beta, state, out=None, qk_l2norm=True, scale=0.0, A_log=None,
+                      dt_bias=None, slot_ids=None, norm_z=None, norm_weight=None, norm_eps=1e-6,
+                      stream=None, check=True):
+    """``recurrent_step`` with any of the fusions of ``gdn_recurrent_step_ex`` (see chunk_fwd_ex)."""
+    import torch
+    N, nqk, dk = q.shape
+    nv, dv = v.shape[1], v.shape[2]
+    if out is None:
+        out = torch.empty((N, nv, dv), dtype=v.dtype, device=v.device)
+    p = make_params(nqk, nv, dk, dv, q.dtype == torch.bfloat16, qk_l2norm, scale)
+    x = make_ext(A_log, dt_bias, slot_ids, state.shape[0] if slot_ids is not None else 0, norm_z,
+                 norm_weight, norm_eps)
+    rc = lib().gdn_recurrent_step_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state), _ptr(out),
+                                     int(N), ctypes.byref(p), ctypes.byref(x), _stream(stream))
+    if check and rc != GDN_OK:
+        raise GdnError(rc, "gdn_recurrent_step_ex")
+    return out
+
+
+def gated_rmsnorm(o, z, weight, eps=1e-6, out=None, stream=None, check=True):
+    """y = o / sqrt(mean(o^2) + eps) * weight * silu(z) over the last axis (``gdn_gated_rmsnorm``).
+
+    o, z [..., D] (bf16 or fp32, same dtype, CUDA, contiguous; D in {64, 128});
+    weight [D] fp32.  ``out`` may be ``o`` (in place).
+    """
+    import torch
+    dim = o.shape[-1]
+    if out is None:
+        out = torch.empty_like(o)
+    rc = lib().gdn_gated_rmsnorm(_ptr(o), _ptr(z), _ptr(weight), float(eps), _ptr(out), int(o.numel() // dim),
+                                 int(dim), DTYPE_BF16 if o.dtype == torch.bfloat16 else DTYPE_F32,
+                                 _stream(stream))
+    if check and rc != GDN_OK:
+        raise GdnError(rc, "gdn_gated_rmsnorm")
     return out

@@ -16,6 +16,10 @@
 // 4 consecutive columns (one 16-byte vector) of DK/RG rows in registers, so
 // every state byte is loaded with a 128-bit streaming load before any
 // arithmetic starts and written back with a 128-bit streaming store.
+//
+// With the gated RMSNorm epilogue (kNorm; RMSNormGated of the walkthrough's
+// sections 一(一)1 and 6) the Dv outputs of the row are normalised in the same
+// CTA before the store: y = o / sqrt(mean(o^2) + eps) * w * silu(z).
 #include "gdn_common.cuh"
 #include "gdn_launch.h"
 
@@ -24,7 +28,7 @@ namespace decode {
 
 constexpr int kThreads = 256;
 
-template <int DK, int DV, typename IO, bool kRawGate>
+template <int DK, int DV, typename IO, bool kRawGate, bool kNorm>
 __global__ void __launch_bounds__(kThreads, 2) recurrent_step_kernel(StepArgs a) {
   constexpr int CG = DV / 4;         // column groups of 4 fp32
   constexpr int RG = kThreads / CG;  // row groups
@@ -35,6 +39,7 @@ __global__ void __launch_bounds__(kThreads, 2) recurrent_step_kernel(StepArgs a)
   __shared__ __align__(16) float delta[DV];
   __shared__ float kq_s;
   __shared__ float gate_s[2];  // exp(g), beta
+  __shared__ float nrm_s[DV / 32];  // per-warp sums of o^2 (kNorm)
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int h = blockIdx.x, n = blockIdx.y;
@@ -51,6 +56,11 @@ __global__ void __launch_bounds__(kThreads, 2) recurrent_step_kernel(StepArgs a)
     load_gate_t<kRawGate>(a, (size_t)n * a.nv + h, h, gv, bv);
     gate_s[0] = expf(gv);
     gate_s[1] = bv;
+  }
+  float zc = 0.f, wc = 0.f, o_keep = 0.f;  // the norm's gate, gain and input of column tid (kNorm)
+  if (kNorm && tid < DV) {
+    zc = to_f32(static_cast<const IO*>(a.nz)[((size_t)n * a.nv + h) * DV + tid]);
+    wc = a.nw[tid];
   }
   float4* st = reinterpret_cast<float4*>(a.state + ((size_t)srow * a.nv + h) * (size_t)DK * DV);
   float4 s[RPT];
@@ -114,9 +124,25 @@ __global__ void __launch_bounds__(kThreads, 2) recurrent_step_kernel(StepArgs a)
     const size_t vo = ((size_t)n * a.nv + h) * DV + c;
     const float dl = bta * (to_f32(static_cast<const IO*>(a.v)[vo]) - kv);
     delta[c] = dl;
-    static_cast<IO*>(a.out)[vo] = from_f32<IO>(fmaf(dl, kq_s, qs));
+    const float o = fmaf(dl, kq_s, qs);
+    if constexpr (kNorm) {
+      const float ss = warp_sum(o * o);
+      if (lane == 0) nrm_s[warp] = ss;
+      o_keep = o;
+    } else {
+      static_cast<IO*>(a.out)[vo] = from_f32<IO>(o);
+    }
   }
   __syncthreads();
+  if constexpr (kNorm) {
+    if (tid < DV) {
+      float ss = 0.f;
+#pragma unroll
+      for (int w = 0; w < DV / 32; ++w) ss += nrm_s[w];
+      const float inv = rsqrtf(ss * (1.f / DV) + a.neps);
+      static_cast<IO*>(a.out)[((size_t)n * a.nv + h) * DV + tid] = from_f32<IO>(o_keep * inv * wc * silu(zc));
+    }
+  }
   const float4 dl = *reinterpret_cast<const float4*>(delta + cg * 4);
 #pragma unroll
   for (int i = 0; i < RPT; ++i) {
@@ -131,10 +157,17 @@ __global__ void __launch_bounds__(kThreads, 2) recurrent_step_kernel(StepArgs a)
 template <int DK, int DV, typename IO>
 static cudaError_t launch_one(const StepArgs& a, cudaStream_t stream) {
   dim3 grid(a.nv, a.num_seqs);
-  if (a.A_log)
-    recurrent_step_kernel<DK, DV, IO, true><<<grid, kThreads, 0, stream>>>(a);
-  else
-    recurrent_step_kernel<DK, DV, IO, false><<<grid, kThreads, 0, stream>>>(a);
+  if (a.nz) {
+    if (a.A_log)
+      recurrent_step_kernel<DK, DV, IO, true, true><<<grid, kThreads, 0, stream>>>(a);
+    else
+      recurrent_step_kernel<DK, DV, IO, false, true><<<grid, kThreads, 0, stream>>>(a);
+  } else {
+    if (a.A_log)
+      recurrent_step_kernel<DK, DV, IO, true, false><<<grid, kThreads, 0, stream>>>(a);
+    else
+      recurrent_step_kernel<DK, DV, IO, false, false><<<grid, kThreads, 0, stream>>>(a);
+  }
   return cudaGetLastError();
 }
 

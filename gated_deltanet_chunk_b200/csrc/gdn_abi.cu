@@ -66,7 +66,7 @@ float resolve_scale(const gdn_params_t* p) {
 
 }  // namespace
 
-GDN_API int gdn_version(void) { return (1 << 16) | 2; }
+GDN_API int gdn_version(void) { return (1 << 16) | 3; }
 
 GDN_API const char* gdn_status_string(int status) {
   switch (status) {
@@ -82,19 +82,38 @@ GDN_API const char* gdn_status_string(int status) {
   }
 }
 
-// Shared by gdn_chunk_fwd (A_log == dt_bias == nullptr: g and beta given) and
-// gdn_chunk_fwd_gated (g, beta slots hold the raw projections a, b).
+// Validates the fusions of an extension block that do not depend on the call.
+static int check_ext(const gdn_ext_t& x) {
+  if ((x.A_log == nullptr) != (x.dt_bias == nullptr)) return GDN_ERR_NULL;
+  if ((x.A_log && !aligned4(x.A_log)) || (x.dt_bias && !aligned4(x.dt_bias))) return GDN_ERR_ALIGN;
+  if (x.slot_ids) {
+    if (x.num_slots < 1) return GDN_ERR_SHAPE;
+    if (!aligned4(x.slot_ids)) return GDN_ERR_ALIGN;
+  }
+  if (x.norm_z) {
+    if (!x.norm_weight) return GDN_ERR_NULL;
+    if (!std::isfinite(x.norm_eps) || x.norm_eps < 0.f) return GDN_ERR_SHAPE;
+    if (!aligned16(x.norm_z) || !aligned16(x.norm_weight)) return GDN_ERR_ALIGN;
+  }
+  return GDN_OK;
+}
+
+// Every chunked-forward entry point lands here; `x` selects the fusions
+// (fused gate: the g, beta slots hold the raw projections a, b; slot pool;
+// gated RMSNorm epilogue).
 static int chunk_fwd_impl(const void* q, const void* k, const void* v, const float* g,
-                          const float* beta, const float* A_log, const float* dt_bias,
-                          const float* initial_state, const int32_t* cu_seqlens, int32_t num_seqs,
-                          int64_t total_tokens, int32_t chunk_size, void* out, float* final_state,
-                          const gdn_params_t* p, void* cuda_stream, const int32_t* slots = nullptr,
-                          int32_t num_slots = 0) {
+                          const float* beta, const float* initial_state, const int32_t* cu_seqlens,
+                          int32_t num_seqs, int64_t total_tokens, int32_t chunk_size, void* out,
+                          float* final_state, const gdn_params_t* p, void* cuda_stream,
+                          const gdn_ext_t& x) {
   int rc = check_params(p);
   if (rc) return rc;
   if (!q || !k || !v || !g || !beta || !out) return GDN_ERR_NULL;
-  if ((A_log == nullptr) != (dt_bias == nullptr)) return GDN_ERR_NULL;
-  if ((A_log && !aligned4(A_log)) || (dt_bias && !aligned4(dt_bias))) return GDN_ERR_ALIGN;
+  rc = check_ext(x);
+  if (rc) return rc;
+  const float *A_log = x.A_log, *dt_bias = x.dt_bias;
+  const int32_t* slots = x.slot_ids;
+  const int32_t num_slots = x.num_slots;
   if (num_seqs < 1 || num_seqs > 65535) return GDN_ERR_SHAPE;
   if (total_tokens < 0 || total_tokens >= (int64_t(1) << 31)) return GDN_ERR_SHAPE;
   if (chunk_size != 64 && chunk_size != 128) return GDN_ERR_SHAPE;
@@ -118,9 +137,11 @@ static int chunk_fwd_impl(const void* q, const void* k, const void* v, const flo
   const Range rsl = slots ? range_of(slots, N * 4) : Range{0, 0};
   const Range ro = range_of(out, T * nv * dv * esz);
   const Range rsf = final_state ? range_of(final_state, rows * nv * dk * dv * 4) : Range{0, 0};
-  for (Range r : {rq, rk, rv, rg, rb, ra, rd, rs0, rcu, rsl, rsf})
+  const Range rz = x.norm_z ? range_of(x.norm_z, T * nv * dv * esz) : Range{0, 0};
+  const Range rw = x.norm_z ? range_of(x.norm_weight, dv * 4) : Range{0, 0};
+  for (Range r : {rq, rk, rv, rg, rb, ra, rd, rs0, rcu, rsl, rsf, rz, rw})
     if (overlap(ro, r)) return GDN_ERR_ALIAS;
-  for (Range r : {rq, rk, rv, rg, rb, ra, rd, rcu, rsl})
+  for (Range r : {rq, rk, rv, rg, rb, ra, rd, rcu, rsl, rz, rw})
     if (overlap(rsf, r)) return GDN_ERR_ALIAS;
   if (final_state && initial_state && (const void*)final_state != (const void*)initial_state &&
       overlap(rsf, rs0))
@@ -138,17 +159,32 @@ static int chunk_fwd_impl(const void* q, const void* k, const void* v, const flo
   a.nqk = p->num_qk_heads; a.nv = p->num_v_heads; a.dv = p->head_v_dim;
   a.qk_l2norm = p->qk_l2norm ? 1 : 0;
   a.scale = resolve_scale(p);
+  a.nz = x.norm_z; a.nw = x.norm_weight; a.neps = x.norm_eps;
   cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
 
   const int bf16 = p->io_dtype == GDN_DTYPE_BF16;
   const bool tc_ok = gdn::chunk_tc_supported(p->head_k_dim, p->head_v_dim, chunk_size, bf16, total_tokens);
   if (p->kernel == GDN_KERNEL_TC && !tc_ok) return GDN_ERR_SHAPE;
+  // Both chunk kernels split Dv across CTAs and store o; the norm epilogue then
+  // rewrites the rows in place (one HBM-bound pass).  Fused into the
+  // tensor-core kernel's output warps it measured slower: those warps also
+  // update rows 64..127 of the state, so their epilogue sits on the serial chain.
+  a.nz = nullptr;
   cudaError_t e;
   if (tc_ok && p->kernel != GDN_KERNEL_SIMT)
     e = gdn::launch_chunk_tc(a, total_tokens, stream);
   else
     e = gdn::launch_chunk_simt(a, p->head_k_dim, chunk_size, bf16, stream);
+  if (e == cudaSuccess && x.norm_z)
+    e = gdn::launch_gated_rmsnorm(out, x.norm_z, x.norm_weight, x.norm_eps, out, total_tokens * (int64_t)nv,
+                                  (int)dv, bf16, stream);
   return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+static gdn_ext_t ext_of(const float* A_log, const float* dt_bias, const int32_t* slots, int32_t num_slots) {
+  gdn_ext_t x{};
+  x.A_log = A_log; x.dt_bias = dt_bias; x.slot_ids = slots; x.num_slots = num_slots;
+  return x;
 }
 
 GDN_API int gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
@@ -156,8 +192,8 @@ GDN_API int gdn_chunk_fwd(const void* q, const void* k, const void* v, const flo
                           const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens,
                           int32_t chunk_size, void* out, float* final_state,
                           const gdn_params_t* p, void* cuda_stream) {
-  return chunk_fwd_impl(q, k, v, g, beta, nullptr, nullptr, initial_state, cu_seqlens, num_seqs,
-                        total_tokens, chunk_size, out, final_state, p, cuda_stream);
+  return chunk_fwd_impl(q, k, v, g, beta, initial_state, cu_seqlens, num_seqs, total_tokens, chunk_size, out,
+                        final_state, p, cuda_stream, ext_of(nullptr, nullptr, nullptr, 0));
 }
 
 GDN_API int gdn_chunk_fwd_slots(const void* q, const void* k, const void* v, const float* g,
@@ -166,10 +202,8 @@ GDN_API int gdn_chunk_fwd_slots(const void* q, const void* k, const void* v, con
                                 int64_t total_tokens, int32_t chunk_size, void* out,
                                 const gdn_params_t* p, void* cuda_stream) {
   if (!state_pool || !slot_ids) return GDN_ERR_NULL;
-  if (num_slots < 1) return GDN_ERR_SHAPE;
-  if (!aligned4(slot_ids)) return GDN_ERR_ALIGN;
-  return chunk_fwd_impl(q, k, v, g, beta, nullptr, nullptr, state_pool, cu_seqlens, num_seqs,
-                        total_tokens, chunk_size, out, state_pool, p, cuda_stream, slot_ids, num_slots);
+  return chunk_fwd_impl(q, k, v, g, beta, state_pool, cu_seqlens, num_seqs, total_tokens, chunk_size, out,
+                        state_pool, p, cuda_stream, ext_of(nullptr, nullptr, slot_ids, num_slots));
 }
 
 GDN_API int gdn_chunk_fwd_gated(const void* q, const void* k, const void* v, const float* a,
@@ -179,20 +213,32 @@ GDN_API int gdn_chunk_fwd_gated(const void* q, const void* k, const void* v, con
                                 void* out, float* final_state, const gdn_params_t* p,
                                 void* cuda_stream) {
   if (!A_log || !dt_bias) return GDN_ERR_NULL;
-  return chunk_fwd_impl(q, k, v, a, b, A_log, dt_bias, initial_state, cu_seqlens, num_seqs,
-                        total_tokens, chunk_size, out, final_state, p, cuda_stream);
+  return chunk_fwd_impl(q, k, v, a, b, initial_state, cu_seqlens, num_seqs, total_tokens, chunk_size, out,
+                        final_state, p, cuda_stream, ext_of(A_log, dt_bias, nullptr, 0));
+}
+
+GDN_API int gdn_chunk_fwd_ex(const void* q, const void* k, const void* v, const float* g,
+                             const float* beta, const float* initial_state, const int32_t* cu_seqlens,
+                             int32_t num_seqs, int64_t total_tokens, int32_t chunk_size, void* out,
+                             float* final_state, const gdn_params_t* p, const gdn_ext_t* ext,
+                             void* cuda_stream) {
+  const gdn_ext_t x = ext ? *ext : gdn_ext_t{};
+  if (x.slot_ids && (!initial_state || final_state != initial_state)) return GDN_ERR_NULL;
+  return chunk_fwd_impl(q, k, v, g, beta, initial_state, cu_seqlens, num_seqs, total_tokens, chunk_size, out,
+                        final_state, p, cuda_stream, x);
 }
 
 static int recurrent_step_impl(const void* q, const void* k, const void* v, const float* g,
-                               const float* beta, const float* A_log, const float* dt_bias,
-                               float* state, void* out, int32_t num_seqs, const gdn_params_t* p,
-                               void* cuda_stream, const int32_t* slots = nullptr,
-                               int32_t num_slots = 0) {
+                               const float* beta, float* state, void* out, int32_t num_seqs,
+                               const gdn_params_t* p, void* cuda_stream, const gdn_ext_t& x) {
   int rc = check_params(p);
   if (rc) return rc;
   if (!q || !k || !v || !g || !beta || !state || !out) return GDN_ERR_NULL;
-  if ((A_log == nullptr) != (dt_bias == nullptr)) return GDN_ERR_NULL;
-  if ((A_log && !aligned4(A_log)) || (dt_bias && !aligned4(dt_bias))) return GDN_ERR_ALIGN;
+  rc = check_ext(x);
+  if (rc) return rc;
+  const float *A_log = x.A_log, *dt_bias = x.dt_bias;
+  const int32_t* slots = x.slot_ids;
+  const int32_t num_slots = x.num_slots;
   if (num_seqs < 1 || num_seqs > 65535) return GDN_ERR_SHAPE;
   const void* ptrs[] = {q, k, v, g, beta, state, out};
   for (const void* ptr : ptrs)
@@ -209,9 +255,11 @@ static int recurrent_step_impl(const void* q, const void* k, const void* v, cons
   const Range rs = range_of(state, (slots ? (size_t)num_slots : N) * nv * dk * dv * 4);
   const Range rsl = slots ? range_of(slots, N * 4) : Range{0, 0};
   const Range ro = range_of(out, N * nv * dv * esz);
-  for (Range r : {rq, rk, rv, rg, rb, ra, rd, rs, rsl})
+  const Range rz = x.norm_z ? range_of(x.norm_z, N * nv * dv * esz) : Range{0, 0};
+  const Range rw = x.norm_z ? range_of(x.norm_weight, dv * 4) : Range{0, 0};
+  for (Range r : {rq, rk, rv, rg, rb, ra, rd, rs, rsl, rz, rw})
     if (overlap(ro, r)) return GDN_ERR_ALIAS;
-  for (Range r : {rq, rk, rv, rg, rb, ra, rd, rsl})
+  for (Range r : {rq, rk, rv, rg, rb, ra, rd, rsl, rz, rw})
     if (overlap(rs, r)) return GDN_ERR_ALIAS;
 
   rc = check_device();
@@ -224,6 +272,7 @@ static int recurrent_step_impl(const void* q, const void* k, const void* v, cons
   a.nqk = p->num_qk_heads; a.nv = p->num_v_heads;
   a.qk_l2norm = p->qk_l2norm ? 1 : 0;
   a.scale = resolve_scale(p);
+  a.nz = x.norm_z; a.nw = x.norm_weight; a.neps = x.norm_eps;
   cudaError_t e = gdn::launch_recurrent_step(a, p->head_k_dim, p->head_v_dim,
                                              p->io_dtype == GDN_DTYPE_BF16,
                                              static_cast<cudaStream_t>(cuda_stream));
@@ -233,7 +282,8 @@ static int recurrent_step_impl(const void* q, const void* k, const void* v, cons
 GDN_API int gdn_recurrent_step(const void* q, const void* k, const void* v, const float* g,
                                const float* beta, float* state, void* out, int32_t num_seqs,
                                const gdn_params_t* p, void* cuda_stream) {
-  return recurrent_step_impl(q, k, v, g, beta, nullptr, nullptr, state, out, num_seqs, p, cuda_stream);
+  return recurrent_step_impl(q, k, v, g, beta, state, out, num_seqs, p, cuda_stream,
+                             ext_of(nullptr, nullptr, nullptr, 0));
 }
 
 GDN_API int gdn_recurrent_step_slots(const void* q, const void* k, const void* v, const float* g,
@@ -241,10 +291,8 @@ GDN_API int gdn_recurrent_step_slots(const void* q, const void* k, const void* v
                                      int32_t num_slots, void* out, int32_t num_seqs,
                                      const gdn_params_t* p, void* cuda_stream) {
   if (!slot_ids) return GDN_ERR_NULL;
-  if (num_slots < 1) return GDN_ERR_SHAPE;
-  if (!aligned4(slot_ids)) return GDN_ERR_ALIGN;
-  return recurrent_step_impl(q, k, v, g, beta, nullptr, nullptr, state_pool, out, num_seqs, p,
-                             cuda_stream, slot_ids, num_slots);
+  return recurrent_step_impl(q, k, v, g, beta, state_pool, out, num_seqs, p, cuda_stream,
+                             ext_of(nullptr, nullptr, slot_ids, num_slots));
 }
 
 GDN_API int gdn_recurrent_step_gated(const void* q, const void* k, const void* v, const float* a,
@@ -252,7 +300,35 @@ GDN_API int gdn_recurrent_step_gated(const void* q, const void* k, const void* v
                                      float* state, void* out, int32_t num_seqs,
                                      const gdn_params_t* p, void* cuda_stream) {
   if (!A_log || !dt_bias) return GDN_ERR_NULL;
-  return recurrent_step_impl(q, k, v, a, b, A_log, dt_bias, state, out, num_seqs, p, cuda_stream);
+  return recurrent_step_impl(q, k, v, a, b, state, out, num_seqs, p, cuda_stream,
+                             ext_of(A_log, dt_bias, nullptr, 0));
+}
+
+GDN_API int gdn_recurrent_step_ex(const void* q, const void* k, const void* v, const float* g,
+                                  const float* beta, float* state, void* out, int32_t num_seqs,
+                                  const gdn_params_t* p, const gdn_ext_t* ext, void* cuda_stream) {
+  return recurrent_step_impl(q, k, v, g, beta, state, out, num_seqs, p, cuda_stream,
+                             ext ? *ext : gdn_ext_t{});
+}
+
+GDN_API int gdn_gated_rmsnorm(const void* o, const void* z, const float* weight, float eps, void* y,
+                              int64_t rows, int32_t dim, int32_t io_dtype, void* cuda_stream) {
+  if (rows < 0 || rows >= (int64_t(1) << 31) || (dim != 64 && dim != 128)) return GDN_ERR_SHAPE;
+  if (io_dtype != GDN_DTYPE_F32 && io_dtype != GDN_DTYPE_BF16) return GDN_ERR_SHAPE;
+  if (!std::isfinite(eps) || eps < 0.f) return GDN_ERR_SHAPE;
+  if (rows == 0) return GDN_OK;  // nothing is read or written
+  if (!o || !z || !weight || !y) return GDN_ERR_NULL;
+  for (const void* ptr : {o, z, (const void*)weight, (const void*)y})
+    if (!aligned16(ptr)) return GDN_ERR_ALIGN;
+  const size_t bytes = (size_t)rows * dim * (io_dtype == GDN_DTYPE_BF16 ? 2 : 4);
+  const Range ry = range_of(y, bytes);
+  if (overlap(ry, range_of(z, bytes)) || overlap(ry, range_of(weight, (size_t)dim * 4))) return GDN_ERR_ALIAS;
+  if (y != o && overlap(ry, range_of(o, bytes))) return GDN_ERR_ALIAS;
+  const int rc = check_device();
+  if (rc) return rc;
+  const cudaError_t e = gdn::launch_gated_rmsnorm(o, z, weight, eps, y, rows, dim, io_dtype == GDN_DTYPE_BF16,
+                                                  static_cast<cudaStream_t>(cuda_stream));
+  return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
 GDN_API int gdn_device_status(void* cuda_stream) {

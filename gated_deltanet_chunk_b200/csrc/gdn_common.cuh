@@ -30,6 +30,9 @@ struct ChunkArgs {
   int32_t nqk, nv, dv;
   int32_t qk_l2norm;
   float scale;
+  const void* nz;            // [T, Nv, Dv] gate of the RMSNorm epilogue, or nullptr (no norm)
+  const float* nw;           // [Dv] RMSNorm gain (with nz)
+  float neps;                // RMSNorm eps (with nz)
 };
 
 // Arguments of the one-token decode step (gdn_recurrent_step).
@@ -49,6 +52,9 @@ struct StepArgs {
   int32_t nqk, nv;
   int32_t qk_l2norm;
   float scale;
+  const void* nz;      // [N, Nv, Dv] gate of the RMSNorm epilogue, or nullptr (no norm)
+  const float* nw;     // [Dv] RMSNorm gain (with nz)
+  float neps;          // RMSNorm eps (with nz)
 };
 
 template <typename T> __device__ __forceinline__ float to_f32(T x);
@@ -110,6 +116,14 @@ __device__ __forceinline__ int64_t state_row(const Args& a, int n) {
   const int32_t s = a.slots[n];
   return (s >= 0 && s < a.num_slots) ? (int64_t)s : -1;
 }
+
+// SiLU, x * sigmoid(x) = x / (1 + exp(-x)): the gate of the RMSNorm epilogue
+// (RMSNormGated of the "手撕Qwen3-Next" walkthrough, sections 一(一)1 and 6)
+// and the activation after the causal conv (section 一(一)3).  Evaluated with
+// the fast intrinsics (a few ulp; the accurate expf and IEEE division made the
+// HBM-bound epilogue instruction-bound); the exponent is clamped at 80 so the
+// divisor stays below the 2^126 limit of __fdividef (silu(-80) is -1.4e-33).
+__device__ __forceinline__ float silu(float x) { return __fdividef(x, 1.f + __expf(fminf(-x, 80.f))); }
 
 // Sequence bounds [start, end) of sequence n.
 __device__ __forceinline__ void seq_bounds(const int32_t* cu, int32_t uniform_len, int n,

@@ -19,4 +19,8 @@ unsigned int chunk_tc_take_status();
 // One-token decode step; dk, dv in {64,128}.
 cudaError_t launch_recurrent_step(const StepArgs& a, int dk, int dv, int io_bf16, cudaStream_t s);
 
+// Gated RMSNorm rows: y = o / sqrt(mean(o^2) + eps) * w * silu(z); dim in {64,128}; y may be o.
+cudaError_t launch_gated_rmsnorm(const void* o, const void* z, const float* w, float eps, void* y,
+                                 int64_t rows, int dim, int io_bf16, cudaStream_t s);
+
 }  // namespace gdn

@@ -191,6 +191,79 @@ int gdn_recurrent_step_gated(const void *q, const void *k, const void *v,
                              const gdn_params_t *p, void *cuda_stream);
 
 /*
+ * gdn_ext_t -- optional fusions around the core, taken by gdn_chunk_fwd_ex and
+ * gdn_recurrent_step_ex.  A NULL pointer or an all-zero struct selects none,
+ * and the _ex calls then equal gdn_chunk_fwd / gdn_recurrent_step.  Fields:
+ *
+ *   A_log, dt_bias   fused gate, as the _gated calls: both non-NULL => the g and
+ *                    beta arguments hold the raw projections a and b.
+ *   slot_ids,        slot pool, as the _slots calls: non-NULL slot_ids => the
+ *   num_slots        state arguments address a pool [num_slots, Nv, Dk, Dv];
+ *                    gdn_chunk_fwd_ex then requires final_state == initial_state
+ *                    (the pool, non-NULL).
+ *   norm_z,          gated RMSNorm epilogue (RMSNormGated of the walkthrough's
+ *   norm_weight,     sections 一(一)1 and 6): non-NULL norm_z => every (token,
+ *   norm_eps         v-head) row o of Dv outputs is stored as
+ *                        y = o / sqrt(mean(o^2) + norm_eps) * norm_weight * silu(z),
+ *                        silu(x) = x / (1 + exp(-x)),
+ *                    computed in fp32.  gdn_recurrent_step_ex normalises the fp32 o
+ *                    before its one rounding to io_dtype; gdn_chunk_fwd_ex stores o
+ *                    and then rewrites each row in place (gdn_gated_rmsnorm), so
+ *                    there o is rounded to io_dtype once before the norm.
+ *                    norm_z has the shape and dtype of `out` ([T or N, Nv, Dv]),
+ *                    norm_weight is [Dv] fp32, both 16-byte aligned and counted as
+ *                    inputs for the overlap rules; norm_eps is finite and >= 0
+ *                    (the layer's default is 1e-6).  A padding slot's decode row
+ *                    stays zero.
+ */
+typedef struct {
+    const float *A_log;
+    const float *dt_bias;
+    const int32_t *slot_ids;
+    int32_t num_slots;
+    const void *norm_z;
+    const float *norm_weight;
+    float norm_eps;
+} gdn_ext_t;
+
+/*
+ * gdn_chunk_fwd_ex / gdn_recurrent_step_ex -- gdn_chunk_fwd / gdn_recurrent_step
+ * with the fusions selected in `ext` (any combination).  Every argument, shape
+ * rule, overlap rule and status code of the plain calls applies; `ext` adds its
+ * own (GDN_ERR_NULL for a half-given gate or a norm_z without norm_weight,
+ * GDN_ERR_SHAPE for num_slots < 1 or a bad norm_eps, GDN_ERR_ALIGN, GDN_ERR_ALIAS
+ * when out overlaps norm_z or norm_weight).
+ */
+int gdn_chunk_fwd_ex(const void *q, const void *k, const void *v,
+                     const float *g, const float *beta,
+                     const float *initial_state,
+                     const int32_t *cu_seqlens,
+                     int32_t num_seqs, int64_t total_tokens, int32_t chunk_size,
+                     void *out, float *final_state,
+                     const gdn_params_t *p, const gdn_ext_t *ext, void *cuda_stream);
+
+int gdn_recurrent_step_ex(const void *q, const void *k, const void *v,
+                          const float *g, const float *beta,
+                          float *state, void *out, int32_t num_seqs,
+                          const gdn_params_t *p, const gdn_ext_t *ext, void *cuda_stream);
+
+/*
+ * gdn_gated_rmsnorm -- the gated RMSNorm epilogue on its own (RMSNormGated,
+ * walkthrough sections 一(一)1 and 6), for rows produced elsewhere:
+ *
+ *   y[r, :] = o[r, :] / sqrt(mean(o[r, :]^2) + eps) * weight * silu(z[r, :])
+ *
+ *   o, z, y   [rows, dim] io_dtype (gdn_dtype_t), 16-byte aligned; y may be o
+ *             (in place) but must not overlap z or weight otherwise
+ *   weight    [dim] fp32, 16-byte aligned
+ *   rows      >= 0 (< 2^31);  dim in {64, 128};  eps finite, >= 0.  With rows == 0
+ *             the call does nothing and returns GDN_OK (the pointers may be NULL).
+ */
+int gdn_gated_rmsnorm(const void *o, const void *z, const float *weight, float eps,
+                      void *y, int64_t rows, int32_t dim, int32_t io_dtype,
+                      void *cuda_stream);
+
+/*
  * gdn_device_status -- synchronise `cuda_stream`, then read and clear the
  * library's device-side error word for the current device.  Returns GDN_OK,
  * GDN_ERR_DEVICE_TIMEOUT if a kernel gave up a bounded wait since the last

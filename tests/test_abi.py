@@ -153,3 +153,63 @@ def test_slots_validation(L):
     import torch
     if not torch.cuda.is_available():
         assert chunk() in (-5, -6)                   # valid: stops at the device check
+
+
+def _chunk_ex(L, p, x, s0=None, sf=None, out=A + 0x5000000):
+    vp = ctypes.c_void_p
+    return L.gdn_chunk_fwd_ex(vp(A), vp(A + 0x1000000), vp(A + 0x2000000), vp(A + 0x3000000),
+                              vp(A + 0x4000000), vp(s0), None, 2, 256, 64, vp(out), vp(sf),
+                              ctypes.byref(p), ctypes.byref(x) if x is not None else None, None)
+
+
+def test_ext_validation(L):
+    import gated_deltanet_chunk_b200 as g
+    import torch
+    p = _p()
+    Z, W = A + 0xA000000, A + 0xB000000
+
+    def ext(**kw):
+        x = g.GdnExt()
+        for k_, v_ in kw.items():
+            setattr(x, k_, v_)
+        return x
+    assert _chunk_ex(L, p, ext(A_log=A + 0x8000000)) == -1                     # half a gate
+    assert _chunk_ex(L, p, ext(norm_z=Z)) == -1                                # norm without weight
+    assert _chunk_ex(L, p, ext(norm_z=Z, norm_weight=W, norm_eps=-1.0)) == -2   # negative eps
+    assert _chunk_ex(L, p, ext(norm_z=Z, norm_weight=W, norm_eps=float("nan"))) == -2
+    assert _chunk_ex(L, p, ext(norm_z=Z + 8, norm_weight=W)) == -3             # 16-byte alignment
+    assert _chunk_ex(L, p, ext(norm_z=Z, norm_weight=W + 4)) == -3
+    assert _chunk_ex(L, p, ext(norm_z=Z, norm_weight=W), out=Z) == -4          # out over z
+    assert _chunk_ex(L, p, ext(norm_z=A + 0x5000000 + 4096, norm_weight=W)) == -4
+    assert _chunk_ex(L, p, ext(slot_ids=A + 0x9000000, num_slots=0),
+                     s0=A + 0x8000000, sf=A + 0x8000000) == -2                 # empty pool
+    assert _chunk_ex(L, p, ext(slot_ids=A + 0x9000000, num_slots=8), s0=A + 0x8000000) == -1  # pool != final
+    vp = ctypes.c_void_p
+    x = ext(norm_z=Z, norm_weight=W)
+    assert L.gdn_recurrent_step_ex(vp(A), vp(A + 0x100000), vp(A + 0x200000), vp(A + 0x300000),
+                                   vp(A + 0x400000), vp(A + 0x500000), vp(Z), 4, ctypes.byref(p),
+                                   ctypes.byref(x), None) == -4                # out over z
+    if not torch.cuda.is_available():
+        assert _chunk_ex(L, p, None) in (-5, -6)                              # NULL ext = plain call
+        assert _chunk_ex(L, p, ext(norm_z=Z, norm_weight=W, norm_eps=1e-6)) in (-5, -6)
+
+
+def test_gated_rmsnorm_validation(L):
+    import torch
+    vp = ctypes.c_void_p
+    O, Z, W, Y = A, A + 0x1000000, A + 0x2000000, A + 0x3000000
+
+    def call(o=O, z=Z, w=W, eps=1e-6, y=Y, rows=100, dim=128, dt=1):
+        return L.gdn_gated_rmsnorm(vp(o), vp(z), vp(w), eps, vp(y), rows, dim, dt, None)
+    assert call(z=None) == -1
+    assert call(o=None, z=None, w=None, y=None, rows=0) == 0   # empty: nothing to do
+    assert call(dim=96) == -2
+    assert call(rows=-1) == -2
+    assert call(dt=7) == -2
+    assert call(eps=-1e-3) == -2
+    assert call(o=O + 2) == -3
+    assert call(y=Z) == -4                    # y over z
+    assert call(y=O + 256) == -4              # y partly over o (in place needs y == o exactly)
+    if not torch.cuda.is_available():
+        assert call(y=O) in (-5, -6)          # in place is valid: stops at the device check
+        assert call() in (-5, -6)

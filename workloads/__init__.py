@@ -181,3 +181,17 @@ def make_decode(num_seqs: int = 256, steps: int = 8, nqk: int = 16, nv: int = 32
                 steps=steps, nqk=nqk, nv=nv, dk=d, dv=d, io=io,
                 a=a.contiguous(), b=b.contiguous(), A_log=torch.log(A.float()).contiguous(),
                 dt_bias=torch.full((nv,), 1.0, device=device))
+
+
+def make_norm_inputs(shape, io: str = "bf16", seed: int = 0, device: str = "cpu"):
+    """Inputs of the gated RMSNorm epilogue for outputs of ``shape`` [..., Dv].
+
+    z ~ N(0, 1) in the io dtype (the layer's z projection of unit-scale hidden
+    states) and a per-column gain ~ U(0.5, 1.5) fp32 (initialised to 1 in the
+    layer; spread here so that a wrong column shows).
+    """
+    gen = torch.Generator(device=device).manual_seed(int(seed) + 7919)
+    dtype = torch.float32 if io == "f32" else torch.bfloat16
+    z = torch.randn(*shape, generator=gen, device=device).to(dtype).contiguous()
+    w = (torch.rand(shape[-1], generator=gen, device=device) + 0.5).contiguous()
+    return z, w
