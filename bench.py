@@ -344,6 +344,21 @@ def run_ours(args, world, rank, local):
                                         call="gdn_gated_rmsnorm", rows=T * nv, dim=D,
                                         gpu_launches=args.steps)
         del z, y
+    # causal conv1d + SiLU producing q, k, v from the packed projection, on the
+    # same tokens (gdn_qkv_conv_fwd with the final conv_state)
+    if not args.no_conv:
+        cv = W.make_conv_inputs(T, nqk, nv, D, D, 4, "bf16", seed=2 + rank, device=str(dev))
+        cq, ck, cvv = torch.empty_like(d["q"]), torch.empty_like(d["k"]), torch.empty_like(d["v"])
+        cst = torch.empty(n, cv["C"], 4, dtype=torch.bfloat16, device=dev)
+
+        def cstep():
+            gdn.qkv_conv_fwd(cv["x"], cv["weight"], nqk, nv, D, D, bias=cv["bias"], num_seqs=n, state_out=cst)
+
+        c_ms = time_steps(cstep, args.warmup, args.steps, stream, world, dev)
+        cb = 2 * T * cv["C"] * 2 + cv["C"] * (4 + 1) * 4 + n * cv["C"] * 4 * 2
+        res["conv"] = hbm_line(c_ms, cb, peaks, peak_src, value=T * world / (c_ms / 1e3), unit="tokens/s",
+                               call="gdn_qkv_conv_fwd", channels=cv["C"], taps=4, gpu_launches=2 * args.steps)
+        del cv, cq, ck, cvv, cst
     # e2e: same call with host buffers (pinned), copies inside the timed region
     if not args.no_e2e:
         hp = {k: host[k].pin_memory() for k in ("q", "k", "v", "g", "beta")}
@@ -476,6 +491,49 @@ def run_decode(args, world, rank, dev, stream, peaks, peak_src):
                                      "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                      "frac": gb / (gms / 1e3) / 1e9 / peaks["hbm_gbs"], "traffic": None,
                                      "peak_source": peak_src, "alg_bytes_per_launch": gb}}
+    if not args.no_conv:
+        # the conv update that produces each step's q, k, v (in-place conv_state), then the step
+        cv = W.make_conv_inputs(wl.num_seqs, wl.nqk, wl.nv, wl.d, wl.d, 4, "bf16", seed=4 + rank,
+                                num_states=wl.num_seqs, device=str(dev))
+        qo, ko, vo = (torch.empty_like(d["q"][0]), torch.empty_like(d["k"][0]), torch.empty_like(d["v"][0]))
+
+        def conv_only():
+            gdn.qkv_conv_update(cv["x"], cv["weight"], cv["state"], wl.nqk, wl.nv, wl.d, wl.d, bias=cv["bias"],
+                                out=(qo, ko, vo))
+
+        it = [0]
+
+        def conv_then_step():
+            conv_only()
+            t = it[0] % steps
+            it[0] += 1
+            gdn.recurrent_step(qo, ko, vo, d["g"][t], d["beta"][t], state, out=out)
+
+        cu_ms = time_steps(conv_only, 32, steps, stream, world, dev)
+        cs_ms = time_steps(conv_then_step, 32, steps, stream, world, dev)
+        C = cv["C"]
+        ub = wl.num_seqs * C * (2 + 2 + 2 * 4 * 2) + C * 5 * 4
+        res["conv_update"] = hbm_line(cu_ms, ub, peaks, peak_src, call="gdn_qkv_conv_update", channels=C,
+                                      gpu_launches=steps)
+        res["conv_then_step"] = hbm_line(cs_ms, byts + ub, peaks, peak_src,
+                                         value=wl.num_seqs * world / (cs_ms / 1e3), unit="tokens/s",
+                                         call="gdn_qkv_conv_update + gdn_recurrent_step", gpu_launches=2 * steps)
+        it[0] = 0
+
+        def conv_fused():
+            t = it[0] % steps
+            it[0] += 1
+            gdn.recurrent_step_ex(None, None, None, d["g"][t], d["beta"][t], state, out=out, conv_x=cv["x"],
+                                  conv_state=cv["state"], conv_weight=cv["weight"], conv_bias=cv["bias"],
+                                  shapes=(wl.nqk, wl.nv, wl.d, wl.d))
+
+        cf_ms = time_steps(conv_fused, 32, steps, stream, world, dev)
+        # the step's bytes without q, k, v, plus the projection, the conv windows and taps
+        qkv = wl.num_seqs * (2 * wl.nqk + wl.nv) * wl.d * 2
+        fb = byts - qkv + wl.num_seqs * C * (2 + 2 * 4 * 2) + C * 5 * 4
+        res["conv_fused"] = hbm_line(cf_ms, fb, peaks, peak_src, value=wl.num_seqs * world / (cf_ms / 1e3),
+                                     unit="tokens/s", call="gdn_recurrent_step_ex (conv_x)", gpu_launches=steps)
+        del cv
     if not args.no_norm:
         z, nw = W.make_norm_inputs((steps, wl.num_seqs, wl.nv, wl.d), "bf16", seed=4 + rank, device=str(dev))
         it = [0]
@@ -541,6 +599,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-gated", action="store_true", help="skip the fused-gate prefill and decode lines")
     ap.add_argument("--no-slots", action="store_true", help="skip the slot-indexed decode line")
+    ap.add_argument("--no-conv", action="store_true",
+                    help="skip the causal-conv lines (prefill conv, decode conv update)")
     ap.add_argument("--no-norm", action="store_true",
                     help="skip the gated-RMSNorm lines (fused prefill and decode, standalone epilogue)")
     ap.add_argument("--no-cpu-baseline", action="store_true")

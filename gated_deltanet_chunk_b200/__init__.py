@@ -15,6 +15,7 @@ chunk_fwd_slots / recurrent_step_slots                         states in a slot-
 chunk_fwd_ex / recurrent_step_ex                               any of those fusions plus the
                                                                gated RMSNorm epilogue (gdn_ext_t)
 gated_rmsnorm(o, z, weight, eps)       -> y                    the epilogue alone, gdn_gated_rmsnorm
+qkv_conv_fwd / qkv_conv_update         -> (q, k, v[, state])  causal conv1d + SiLU producing q, k, v
 """
 from __future__ import annotations
 
@@ -48,7 +49,9 @@ class GdnParams(ctypes.Structure):
 class GdnExt(ctypes.Structure):
     _fields_ = [("A_log", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p), ("slot_ids", ctypes.c_void_p),
                 ("num_slots", ctypes.c_int32), ("norm_z", ctypes.c_void_p), ("norm_weight", ctypes.c_void_p),
-                ("norm_eps", ctypes.c_float)]
+                ("norm_eps", ctypes.c_float), ("conv_x", ctypes.c_void_p), ("conv_state", ctypes.c_void_p),
+                ("conv_weight", ctypes.c_void_p), ("conv_bias", ctypes.c_void_p),
+                ("conv_kernel_size", ctypes.c_int32)]
 
 
 _lib = None
@@ -93,6 +96,12 @@ def lib() -> ctypes.CDLL:
         L.gdn_gated_rmsnorm.argtypes = [vp, vp, fp, ctypes.c_float, vp, ctypes.c_int64, ctypes.c_int32,
                                         ctypes.c_int32, vp]
         L.gdn_gated_rmsnorm.restype = ctypes.c_int
+        L.gdn_qkv_conv_fwd.argtypes = [vp, fp, fp, vp, ip, ctypes.c_int32, ctypes.c_int64, ctypes.c_int32,
+                                       vp, vp, vp, vp, ctypes.POINTER(GdnParams), vp]
+        L.gdn_qkv_conv_fwd.restype = ctypes.c_int
+        L.gdn_qkv_conv_update.argtypes = [vp, fp, fp, vp, ip, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                          vp, vp, vp, ctypes.POINTER(GdnParams), vp]
+        L.gdn_qkv_conv_update.restype = ctypes.c_int
         L.gdn_device_status.argtypes = [vp]
         L.gdn_device_status.restype = ctypes.c_int
         L.gdn_status_string.argtypes = [ctypes.c_int]
@@ -246,11 +255,12 @@ def recurrent_step_slots(q, k, v, g, beta, state_pool, slot_ids, out=None, qk_l2
 
 
 def make_ext(A_log=None, dt_bias=None, slot_ids=None, num_slots=0, norm_z=None, norm_weight=None,
-             norm_eps=1e-6) -> GdnExt:
-    """The gdn_ext_t block: fused gate, slot pool and gated RMSNorm epilogue (each optional)."""
+             norm_eps=1e-6, conv_x=None, conv_state=None, conv_weight=None, conv_bias=None) -> GdnExt:
+    """The gdn_ext_t block: fused gate, slot pool, gated RMSNorm epilogue, fused conv (each optional)."""
     p = lambda t: None if t is None else t.data_ptr()
     return GdnExt(p(A_log), p(dt_bias), p(slot_ids), int(num_slots), p(norm_z), p(norm_weight),
-                  float(norm_eps))
+                  float(norm_eps), p(conv_x), p(conv_state), p(conv_weight), p(conv_bias),
+                  int(conv_weight.shape[1]) if conv_weight is not None else 0)
 
 
 def chunk_fwd_ex(q, k, v, g, beta, initial_state=None, cu_seqlens=None, chunk_size=64, out=None,
@@ -290,16 +300,28 @@ def chunk_fwd_ex(q, k, v, g, beta, initial_state=None, cu_seqlens=None, chunk_si
 
 def recurrent_step_ex(q, k, v, g, beta, state, out=None, qk_l2norm=True, scale=0.0, A_log=None,
                       dt_bias=None, slot_ids=None, norm_z=None, norm_weight=None, norm_eps=1e-6,
+                      conv_x=None, conv_state=None, conv_weight=None, conv_bias=None, shapes=None,
                       stream=None, check=True):
-    """``recurrent_step`` with any of the fusions of ``gdn_recurrent_step_ex`` (see chunk_fwd_ex)."""
+    """``recurrent_step`` with any of the fusions of ``gdn_recurrent_step_ex`` (see chunk_fwd_ex).
+
+    With the conv fused, pass q = k = v = None, ``conv_x`` [N, C], ``conv_state``
+    [N or P, C, K] (updated in place), ``conv_weight`` [C, K], ``conv_bias`` and
+    ``shapes=(nqk, nv, dk, dv)``.
+    """
     import torch
-    N, nqk, dk = q.shape
-    nv, dv = v.shape[1], v.shape[2]
+    if conv_x is not None:
+        nqk, nv, dk, dv = shapes
+        N = conv_x.shape[0]
+        io_bf16, dev = conv_x.dtype == torch.bfloat16, conv_x.device
+    else:
+        N, nqk, dk = q.shape
+        nv, dv = v.shape[1], v.shape[2]
+        io_bf16, dev = q.dtype == torch.bfloat16, v.device
     if out is None:
-        out = torch.empty((N, nv, dv), dtype=v.dtype, device=v.device)
-    p = make_params(nqk, nv, dk, dv, q.dtype == torch.bfloat16, qk_l2norm, scale)
+        out = torch.empty((N, nv, dv), dtype=torch.bfloat16 if io_bf16 else torch.float32, device=dev)
+    p = make_params(nqk, nv, dk, dv, io_bf16, qk_l2norm, scale)
     x = make_ext(A_log, dt_bias, slot_ids, state.shape[0] if slot_ids is not None else 0, norm_z,
-                 norm_weight, norm_eps)
+                 norm_weight, norm_eps, conv_x, conv_state, conv_weight, conv_bias)
     rc = lib().gdn_recurrent_step_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state), _ptr(out),
                                      int(N), ctypes.byref(p), ctypes.byref(x), _stream(stream))
     if check and rc != GDN_OK:
@@ -323,3 +345,55 @@ def gated_rmsnorm(o, z, weight, eps=1e-6, out=None, stream=None, check=True):
     if check and rc != GDN_OK:
         raise GdnError(rc, "gdn_gated_rmsnorm")
     return out
+
+
+def _qkv_out(rows, nqk, nv, dk, dv, dtype, device):
+    import torch
+    return (torch.empty((rows, nqk, dk), dtype=dtype, device=device),
+            torch.empty((rows, nqk, dk), dtype=dtype, device=device),
+            torch.empty((rows, nv, dv), dtype=dtype, device=device))
+
+
+def qkv_conv_fwd(mixed_qkv, weight, nqk, nv, dk, dv, bias=None, conv_state=None, cu_seqlens=None,
+                 num_seqs=None, output_state=True, state_out=None, stream=None, check=True):
+    """Causal depthwise conv1d + SiLU of packed [q | k | v] channels (``gdn_qkv_conv_fwd``).
+
+    mixed_qkv [T, C] (bf16 or fp32), weight [C, K] fp32, bias [C] fp32 or None,
+    conv_state [N, C, K] or None (zeros).  Returns ``(q, k, v, state)`` with q, k
+    [T, Nqk, Dk], v [T, Nv, Dv] and the new conv_state [N, C, K] (None unless
+    requested; ``state_out=conv_state`` updates it in place).
+    """
+    import torch
+    T, C = mixed_qkv.shape
+    K = weight.shape[1]
+    n = (cu_seqlens.numel() - 1) if cu_seqlens is not None else (num_seqs or 1)
+    q, k, v = _qkv_out(T, nqk, nv, dk, dv, mixed_qkv.dtype, mixed_qkv.device)
+    if state_out is None and output_state:
+        state_out = torch.empty((n, C, K), dtype=mixed_qkv.dtype, device=mixed_qkv.device)
+    p = make_params(nqk, nv, dk, dv, mixed_qkv.dtype == torch.bfloat16)
+    rc = lib().gdn_qkv_conv_fwd(_ptr(mixed_qkv), _ptr(weight), _ptr(bias), _ptr(conv_state), _ptr(cu_seqlens),
+                                int(n), int(T), int(K), _ptr(q), _ptr(k), _ptr(v), _ptr(state_out),
+                                ctypes.byref(p), _stream(stream))
+    if check and rc != GDN_OK:
+        raise GdnError(rc, "gdn_qkv_conv_fwd")
+    return q, k, v, state_out
+
+
+def qkv_conv_update(mixed_qkv, weight, conv_state, nqk, nv, dk, dv, bias=None, slot_ids=None, out=None,
+                    stream=None, check=True):
+    """One decode token per sequence through the conv (``gdn_qkv_conv_update``); conv_state in place.
+
+    mixed_qkv [N, C]; conv_state [N, C, K] (or a pool [P, C, K] with slot_ids [N] int32).
+    Returns ``(q, k, v)`` with q, k [N, Nqk, Dk] and v [N, Nv, Dv].
+    """
+    import torch
+    N, C = mixed_qkv.shape
+    K = weight.shape[1]
+    q, k, v = out if out is not None else _qkv_out(N, nqk, nv, dk, dv, mixed_qkv.dtype, mixed_qkv.device)
+    p = make_params(nqk, nv, dk, dv, mixed_qkv.dtype == torch.bfloat16)
+    rc = lib().gdn_qkv_conv_update(_ptr(mixed_qkv), _ptr(weight), _ptr(bias), _ptr(conv_state), _ptr(slot_ids),
+                                   int(conv_state.shape[0]) if slot_ids is not None else 0, int(N), int(K),
+                                   _ptr(q), _ptr(k), _ptr(v), ctypes.byref(p), _stream(stream))
+    if check and rc != GDN_OK:
+        raise GdnError(rc, "gdn_qkv_conv_update")
+    return q, k, v

@@ -1,0 +1,315 @@
+// causal_conv.cu -- causal depthwise conv1d + SiLU of the packed q|k|v channels.
+//
+// The "手撕Qwen3-Next" walkthrough, section 一(一)3 (qkv 卷积部分): every channel
+// of mixed_qkv = [q | k | v] is convolved on its own with K taps, zero padded by
+// K - 1 on the left and cut to the sequence (a causal cross-correlation), then
+// passed through SiLU:
+//
+//   y[t, c] = silu(bias[c] + sum_i w[c, i] * in(t - (K - 1) + i))
+//
+// where in(p) is the input at position p of the sequence, or, for p < 0, the
+// cached window before it (conv_state[n, c, K + p]; zeros without one).  The
+// decode update (torch_causal_conv1d_update) is the same formula over
+// [conv_state, x] for one token, and the new conv_state is the last K inputs.
+//
+// The outputs go straight to the three tensors the chunk and decode kernels
+// read: channels [0, Nqk Dk) to q [T, Nqk, Dk], [Nqk Dk, 2 Nqk Dk) to k, the
+// rest to v [T, Nv, Dv].  Every kernel here is bound by HBM: x is read once
+// and q, k, v written once (the K - 1 earlier rows a thread re-reads are L1
+// hits).  A thread owns one 16-byte vector of channels (8 bf16 or 4 fp32).
+#include "gdn_common.cuh"
+#include "gdn_launch.h"
+
+namespace gdn {
+namespace conv {
+
+constexpr int kThreads = 256;
+constexpr int kTokensPerBlock = 32;  // prefill: consecutive tokens per thread
+
+template <typename IO> struct V16;
+template <> struct V16<float> {
+  static constexpr int N = 4;
+  __device__ static void load(const void* p, float* x) {
+    const float4 v = *reinterpret_cast<const float4*>(p);
+    x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+  }
+  __device__ static void store(void* p, const float* x) {
+    *reinterpret_cast<float4*>(p) = make_float4(x[0], x[1], x[2], x[3]);
+  }
+};
+template <> struct V16<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ static void load(const void* p, float* x) {
+    const uint4 v = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      x[2 * i] = __uint_as_float(w[i] << 16);
+      x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  }
+  __device__ static void store(void* p, const float* x) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+      w[i] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+};
+
+// Raw 16-byte vectors, unpacked to fp32 when used.
+__device__ __forceinline__ uint4 ld16(const void* p) { return *reinterpret_cast<const uint4*>(p); }
+template <typename IO> __device__ __forceinline__ void unpack16(uint4 v, float* x);
+template <> __device__ __forceinline__ void unpack16<float>(uint4 v, float* x) {
+  x[0] = __uint_as_float(v.x); x[1] = __uint_as_float(v.y); x[2] = __uint_as_float(v.z); x[3] = __uint_as_float(v.w);
+}
+template <> __device__ __forceinline__ void unpack16<__nv_bfloat16>(uint4 v, float* x) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    x[2 * i] = __uint_as_float(w[i] << 16);
+    x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+// The taps and bias of channels [c0, c0 + E): w[i][e], b[e] (16-byte loads; the
+// E * K weights of a thread are contiguous and 16-byte aligned).
+template <int E, int K>
+__device__ __forceinline__ void load_taps(const ConvArgs& a, int c0, float (&w)[K][E], float (&b)[E]) {
+  const float4* wp = reinterpret_cast<const float4*>(a.weight + (size_t)c0 * K);
+#pragma unroll
+  for (int q = 0; q < E * K / 4; ++q) {
+    const float4 v = __ldg(wp + q);
+    const float f[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int r = 0; r < 4; ++r) w[(4 * q + r) % K][(4 * q + r) / K] = f[r];
+  }
+#pragma unroll
+  for (int e = 0; e < E; ++e) b[e] = a.bias ? __ldg(a.bias + c0 + e) : 0.f;
+}
+
+// Destination of channel vector c0 (E channels starting at c0) for row t.
+template <typename IO>
+__device__ __forceinline__ IO* out_ptr(const ConvArgs& a, int64_t t, int c0) {
+  const int qk = a.nqk * a.dk;
+  if (c0 < qk) return static_cast<IO*>(a.q) + (size_t)t * qk + c0;
+  if (c0 < 2 * qk) return static_cast<IO*>(a.k) + (size_t)t * qk + (c0 - qk);
+  const int vd = a.nv * a.dv;
+  return static_cast<IO*>(a.v) + (size_t)t * vd + (c0 - 2 * qk);
+}
+
+// Channel c of the window before sequence n: conv_state[row, c, j], j in [0, K).
+template <typename IO>
+__device__ __forceinline__ float window_at(const ConvArgs& a, int64_t row, int c, int j) {
+  if (a.state_in == nullptr || row < 0) return 0.f;
+  return to_f32(static_cast<const IO*>(a.state_in)[((size_t)row * a.channels + c) * a.ksize + j]);
+}
+
+// Sequence of token t (cu is non-decreasing; the first n with cu[n+1] > t).
+__device__ __forceinline__ int seq_of(const int32_t* cu, int num_seqs, int64_t t) {
+  int lo = 0, hi = num_seqs - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if ((int64_t)cu[mid + 1] > t) hi = mid; else lo = mid + 1;
+  }
+  return lo;
+}
+
+// Prefill: block (token block, channel block); thread = one channel vector over
+// kTokensPerBlock consecutive tokens, which may cross sequence boundaries.  The
+// K - 1 previous inputs stay in registers (a sliding window); the rows of the
+// next kBatch tokens are loaded before any of them is used.
+constexpr int kBatch = 8;
+
+template <typename IO, int K>
+__global__ void __launch_bounds__(kThreads) conv_fwd_kernel(ConvArgs a) {
+  constexpr int E = V16<IO>::N;
+  const int c0 = (blockIdx.y * kThreads + threadIdx.x) * E;
+  if (c0 >= a.channels) return;
+  const int64_t t_begin = (int64_t)blockIdx.x * kTokensPerBlock;
+  const int64_t t_end = min((int64_t)a.total_tokens, t_begin + kTokensPerBlock);
+  if (t_begin >= t_end) return;
+  float w[K][E], b[E];
+  load_taps<E, K>(a, c0, w, b);
+  const IO* x = static_cast<const IO*>(a.x);
+  int n = a.cu ? seq_of(a.cu, a.num_seqs, t_begin) : (int)(t_begin / a.uniform_len);
+  int64_t s_begin, s_end;
+  seq_bounds(a.cu, a.uniform_len, n, s_begin, s_end);
+  // win[j] = input at position t - (K - 1) + j for the next token t
+  float win[K > 1 ? K - 1 : 1][E];
+#pragma unroll
+  for (int j = 0; j + 1 < K; ++j) {
+    const int64_t p = t_begin - (K - 1) + j;
+    if (p >= s_begin) {
+      unpack16<IO>(ld16(x + (size_t)p * a.channels + c0), win[j]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < E; ++e) win[j][e] = window_at<IO>(a, n, c0 + e, (int)(K + (p - s_begin)));
+    }
+  }
+  for (int64_t t0 = t_begin; t0 < t_end; t0 += kBatch) {
+    uint4 raw[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u)
+      raw[u] = (t0 + u < t_end) ? ld16(x + (size_t)(t0 + u) * a.channels + c0) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int64_t t = t0 + u;
+      if (t >= t_end) break;
+      if (t >= s_end) {  // first token of the next non-empty sequence: restart the window
+        do {
+          ++n;
+          seq_bounds(a.cu, a.uniform_len, n, s_begin, s_end);
+        } while (t >= s_end);
+#pragma unroll
+        for (int j = 0; j + 1 < K; ++j)
+#pragma unroll
+          for (int e = 0; e < E; ++e) win[j][e] = window_at<IO>(a, n, c0 + e, j + 1);
+      }
+      float xt[E], acc[E];
+      unpack16<IO>(raw[u], xt);
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        float s_ = b[e];
+#pragma unroll
+        for (int j = 0; j + 1 < K; ++j) s_ = fmaf(w[j][e], win[j][e], s_);
+        acc[e] = silu(fmaf(w[K - 1][e], xt[e], s_));
+      }
+      V16<IO>::store(out_ptr<IO>(a, t, c0), acc);
+#pragma unroll
+      for (int j = 0; j + 2 < K; ++j)
+#pragma unroll
+        for (int e = 0; e < E; ++e) win[j][e] = win[j + 1][e];
+      if (K > 1) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) win[K > 1 ? K - 2 : 0][e] = xt[e];
+      }
+    }
+  }
+}
+
+// The conv_state after a prefill: the last K inputs of [window, sequence] of
+// every sequence (thread = one channel of one sequence).  Runs after
+// conv_fwd_kernel on the same stream, so state_out may be state_in.
+template <typename IO, int K>
+__global__ void __launch_bounds__(kThreads) conv_state_kernel(ConvArgs a) {
+  const int64_t idx = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  if (idx >= (int64_t)a.num_seqs * a.channels) return;
+  const int n = (int)(idx / a.channels), c = (int)(idx % a.channels);
+  int64_t s_begin, s_end;
+  seq_bounds(a.cu, a.uniform_len, n, s_begin, s_end);
+  const int64_t len = s_end - s_begin;
+  float v[K];
+#pragma unroll
+  for (int i = 0; i < K; ++i) {
+    const int64_t p = len - K + i;  // position in the sequence
+    v[i] = p >= 0 ? to_f32(static_cast<const IO*>(a.x)[(size_t)(s_begin + p) * a.channels + c])
+                  : window_at<IO>(a, n, c, (int)(K + p));
+  }
+  IO* dst = static_cast<IO*>(a.state_out) + ((size_t)n * a.channels + c) * K;
+#pragma unroll
+  for (int i = 0; i < K; ++i) dst[i] = from_f32<IO>(v[i]);
+}
+
+// Decode: one token per sequence, conv_state updated in place (optionally
+// through slot ids).  Thread = one channel vector of one sequence; its state
+// span (E channels x K taps, 16 K bytes) and its taps move as 16-byte vectors.
+template <typename IO, int K>
+__global__ void __launch_bounds__(kThreads) conv_update_kernel(ConvArgs a) {
+  constexpr int E = V16<IO>::N;
+  constexpr int PER = 16 / (int)sizeof(IO);  // state elements per 16-byte vector
+  const int c0 = (blockIdx.x * kThreads + threadIdx.x) * E;
+  const int n = blockIdx.y;
+  if (c0 >= a.channels) return;
+  int64_t row = n;
+  if (a.slots) {
+    const int32_t s = a.slots[n];
+    row = (s >= 0 && s < a.num_slots) ? s : -1;
+  }
+  float out[E];
+  if (row < 0) {  // a padding sequence: zero output, no state
+#pragma unroll
+    for (int e = 0; e < E; ++e) out[e] = 0.f;
+    V16<IO>::store(out_ptr<IO>(a, n, c0), out);
+    return;
+  }
+  const uint4 xr = ld16(static_cast<const IO*>(a.x) + (size_t)n * a.channels + c0);
+  IO* st = static_cast<IO*>(a.state_out) + ((size_t)row * a.channels + c0) * K;
+  uint4 sr[K];  // E * K state elements, channel-major: element (e, i) at e * K + i
+#pragma unroll
+  for (int q = 0; q < K; ++q) sr[q] = ld16(st + q * PER);
+  float w[K][E], b[E];
+  load_taps<E, K>(a, c0, w, b);
+  float x[E], win[E * K];
+  unpack16<IO>(xr, x);
+#pragma unroll
+  for (int q = 0; q < K; ++q) unpack16<IO>(sr[q], win + q * PER);
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    // taps 0..K-2 meet the window's entries 1..K-1, tap K-1 the new input
+    float acc = b[e];
+#pragma unroll
+    for (int i = 0; i + 1 < K; ++i) acc = fmaf(w[i][e], win[e * K + i + 1], acc);
+    out[e] = silu(fmaf(w[K - 1][e], x[e], acc));
+  }
+  // the new window: shifted by one, the new input last
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+#pragma unroll
+    for (int i = 0; i + 1 < K; ++i) win[e * K + i] = win[e * K + i + 1];
+    win[e * K + K - 1] = x[e];
+  }
+#pragma unroll
+  for (int q = 0; q < K; ++q) V16<IO>::store(st + q * PER, win + q * PER);
+  V16<IO>::store(out_ptr<IO>(a, n, c0), out);
+}
+
+template <typename IO, int K>
+static cudaError_t launch_fwd(const ConvArgs& a, cudaStream_t s) {
+  constexpr int E = V16<IO>::N;
+  const int vecs = a.channels / E;
+  if (a.total_tokens > 0) {
+    dim3 grid((unsigned)((a.total_tokens + kTokensPerBlock - 1) / kTokensPerBlock), (vecs + kThreads - 1) / kThreads);
+    conv_fwd_kernel<IO, K><<<grid, kThreads, 0, s>>>(a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (a.state_out) {
+    const int64_t thr = (int64_t)a.num_seqs * a.channels;
+    conv_state_kernel<IO, K><<<(unsigned)((thr + kThreads - 1) / kThreads), kThreads, 0, s>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+template <typename IO, int K>
+static cudaError_t launch_update(const ConvArgs& a, cudaStream_t s) {
+  constexpr int E = V16<IO>::N;
+  dim3 grid((a.channels / E + kThreads - 1) / kThreads, a.num_seqs);
+  conv_update_kernel<IO, K><<<grid, kThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+template <typename IO>
+static cudaError_t dispatch(const ConvArgs& a, bool update, cudaStream_t s) {
+  switch (a.ksize) {
+    case 1: return update ? launch_update<IO, 1>(a, s) : launch_fwd<IO, 1>(a, s);
+    case 2: return update ? launch_update<IO, 2>(a, s) : launch_fwd<IO, 2>(a, s);
+    case 3: return update ? launch_update<IO, 3>(a, s) : launch_fwd<IO, 3>(a, s);
+    case 4: return update ? launch_update<IO, 4>(a, s) : launch_fwd<IO, 4>(a, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace conv
+
+cudaError_t launch_conv_fwd(const ConvArgs& a, int io_bf16, cudaStream_t s) {
+  return io_bf16 ? conv::dispatch<__nv_bfloat16>(a, false, s) : conv::dispatch<float>(a, false, s);
+}
+
+cudaError_t launch_conv_update(const ConvArgs& a, int io_bf16, cudaStream_t s) {
+  return io_bf16 ? conv::dispatch<__nv_bfloat16>(a, true, s) : conv::dispatch<float>(a, true, s);
+}
+
+}  // namespace gdn

@@ -66,7 +66,7 @@ float resolve_scale(const gdn_params_t* p) {
 
 }  // namespace
 
-GDN_API int gdn_version(void) { return (1 << 16) | 3; }
+GDN_API int gdn_version(void) { return (1 << 16) | 4; }
 
 GDN_API const char* gdn_status_string(int status) {
   switch (status) {
@@ -95,6 +95,13 @@ static int check_ext(const gdn_ext_t& x) {
     if (!std::isfinite(x.norm_eps) || x.norm_eps < 0.f) return GDN_ERR_SHAPE;
     if (!aligned16(x.norm_z) || !aligned16(x.norm_weight)) return GDN_ERR_ALIGN;
   }
+  if (x.conv_x) {
+    if (!x.conv_state || !x.conv_weight) return GDN_ERR_NULL;
+    if (x.conv_kernel_size < 1 || x.conv_kernel_size > 4) return GDN_ERR_SHAPE;
+    if (!aligned16(x.conv_x) || !aligned16(x.conv_state) || !aligned4(x.conv_weight) ||
+        (x.conv_bias && !aligned4(x.conv_bias)))
+      return GDN_ERR_ALIGN;
+  }
   return GDN_OK;
 }
 
@@ -111,6 +118,7 @@ static int chunk_fwd_impl(const void* q, const void* k, const void* v, const flo
   if (!q || !k || !v || !g || !beta || !out) return GDN_ERR_NULL;
   rc = check_ext(x);
   if (rc) return rc;
+  if (x.conv_x) return GDN_ERR_SHAPE;  // the prefill conv is gdn_qkv_conv_fwd
   const float *A_log = x.A_log, *dt_bias = x.dt_bias;
   const int32_t* slots = x.slot_ids;
   const int32_t num_slots = x.num_slots;
@@ -233,16 +241,23 @@ static int recurrent_step_impl(const void* q, const void* k, const void* v, cons
                                const gdn_params_t* p, void* cuda_stream, const gdn_ext_t& x) {
   int rc = check_params(p);
   if (rc) return rc;
-  if (!q || !k || !v || !g || !beta || !state || !out) return GDN_ERR_NULL;
   rc = check_ext(x);
   if (rc) return rc;
+  const bool conv = x.conv_x != nullptr;
+  if (conv) {
+    if (q || k || v) return GDN_ERR_SHAPE;  // the fused conv produces them
+    if (p->num_v_heads / p->num_qk_heads > 8) return GDN_ERR_SHAPE;  // one cluster per qk group
+  } else if (!q || !k || !v) {
+    return GDN_ERR_NULL;
+  }
+  if (!g || !beta || !state || !out) return GDN_ERR_NULL;
   const float *A_log = x.A_log, *dt_bias = x.dt_bias;
   const int32_t* slots = x.slot_ids;
   const int32_t num_slots = x.num_slots;
   if (num_seqs < 1 || num_seqs > 65535) return GDN_ERR_SHAPE;
   const void* ptrs[] = {q, k, v, g, beta, state, out};
   for (const void* ptr : ptrs)
-    if (!aligned16(ptr)) return GDN_ERR_ALIGN;
+    if (ptr && !aligned16(ptr)) return GDN_ERR_ALIGN;
   const size_t N = (size_t)num_seqs;
   const size_t esz = p->io_dtype == GDN_DTYPE_BF16 ? 2 : 4;
   const size_t dk = p->head_k_dim, dv = p->head_v_dim;
@@ -257,10 +272,17 @@ static int recurrent_step_impl(const void* q, const void* k, const void* v, cons
   const Range ro = range_of(out, N * nv * dv * esz);
   const Range rz = x.norm_z ? range_of(x.norm_z, N * nv * dv * esz) : Range{0, 0};
   const Range rw = x.norm_z ? range_of(x.norm_weight, dv * 4) : Range{0, 0};
-  for (Range r : {rq, rk, rv, rg, rb, ra, rd, rs, rsl, rz, rw})
+  const size_t C = 2 * nqk * dk + nv * dv, CK = (size_t)x.conv_kernel_size;
+  const Range rcx = conv ? range_of(x.conv_x, N * C * esz) : Range{0, 0};
+  const Range rcs = conv ? range_of(x.conv_state, (slots ? (size_t)num_slots : N) * C * CK * esz) : Range{0, 0};
+  const Range rcw = conv ? range_of(x.conv_weight, C * CK * 4) : Range{0, 0};
+  const Range rcb = conv && x.conv_bias ? range_of(x.conv_bias, C * 4) : Range{0, 0};
+  for (Range r : {rq, rk, rv, rg, rb, ra, rd, rs, rsl, rz, rw, rcx, rcs, rcw, rcb})
     if (overlap(ro, r)) return GDN_ERR_ALIAS;
-  for (Range r : {rq, rk, rv, rg, rb, ra, rd, rsl, rz, rw})
+  for (Range r : {rq, rk, rv, rg, rb, ra, rd, rsl, rz, rw, rcx, rcs, rcw, rcb})
     if (overlap(rs, r)) return GDN_ERR_ALIAS;
+  for (Range r : {rg, rb, ra, rd, rsl, rz, rw, rcx, rcw, rcb})
+    if (overlap(rcs, r)) return GDN_ERR_ALIAS;
 
   rc = check_device();
   if (rc) return rc;
@@ -273,6 +295,8 @@ static int recurrent_step_impl(const void* q, const void* k, const void* v, cons
   a.qk_l2norm = p->qk_l2norm ? 1 : 0;
   a.scale = resolve_scale(p);
   a.nz = x.norm_z; a.nw = x.norm_weight; a.neps = x.norm_eps;
+  a.cx = x.conv_x; a.cstate = x.conv_state; a.cw = x.conv_weight; a.cb = x.conv_bias;
+  a.cks = x.conv_kernel_size;
   cudaError_t e = gdn::launch_recurrent_step(a, p->head_k_dim, p->head_v_dim,
                                              p->io_dtype == GDN_DTYPE_BF16,
                                              static_cast<cudaStream_t>(cuda_stream));
@@ -328,6 +352,101 @@ GDN_API int gdn_gated_rmsnorm(const void* o, const void* z, const float* weight,
   if (rc) return rc;
   const cudaError_t e = gdn::launch_gated_rmsnorm(o, z, weight, eps, y, rows, dim, io_dtype == GDN_DTYPE_BF16,
                                                   static_cast<cudaStream_t>(cuda_stream));
+  return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+// Shared validation of the two conv calls; fills the launch block.
+static int conv_common(const void* x, const float* weight, const float* bias, int32_t kernel_size, void* q,
+                       void* k, void* v, int32_t num_seqs, const gdn_params_t* p, gdn::ConvArgs& a) {
+  int rc = check_params(p);
+  if (rc) return rc;
+  if (!x || !weight || !q || !k || !v) return GDN_ERR_NULL;
+  if (kernel_size < 1 || kernel_size > 4) return GDN_ERR_SHAPE;
+  if (num_seqs < 1 || num_seqs > 65535) return GDN_ERR_SHAPE;
+  for (const void* ptr : {x, (const void*)q, (const void*)k, (const void*)v})
+    if (!aligned16(ptr)) return GDN_ERR_ALIGN;
+  if (!aligned4(weight) || (bias && !aligned4(bias))) return GDN_ERR_ALIGN;
+  a = gdn::ConvArgs{};
+  a.x = x; a.weight = weight; a.bias = bias; a.num_seqs = num_seqs; a.ksize = kernel_size;
+  a.nqk = p->num_qk_heads; a.nv = p->num_v_heads; a.dk = p->head_k_dim; a.dv = p->head_v_dim;
+  a.channels = 2 * a.nqk * a.dk + a.nv * a.dv;
+  a.q = q; a.k = k; a.v = v;
+  return GDN_OK;
+}
+
+GDN_API int gdn_qkv_conv_fwd(const void* mixed_qkv, const float* weight, const float* bias,
+                             const void* conv_state_in, const int32_t* cu_seqlens, int32_t num_seqs,
+                             int64_t total_tokens, int32_t kernel_size, void* q, void* k, void* v,
+                             void* conv_state_out, const gdn_params_t* p, void* cuda_stream) {
+  gdn::ConvArgs a;
+  int rc = conv_common(mixed_qkv, weight, bias, kernel_size, q, k, v, num_seqs, p, a);
+  if (rc) return rc;
+  if (total_tokens < 0 || total_tokens >= (int64_t(1) << 31)) return GDN_ERR_SHAPE;
+  if (!cu_seqlens && total_tokens % num_seqs != 0) return GDN_ERR_SHAPE;
+  for (const void* ptr : {conv_state_in, (const void*)conv_state_out, (const void*)cu_seqlens})
+    if (ptr && !aligned16(ptr)) return GDN_ERR_ALIGN;
+  const size_t T = (size_t)total_tokens, N = (size_t)num_seqs, C = (size_t)a.channels, K = kernel_size;
+  const size_t esz = p->io_dtype == GDN_DTYPE_BF16 ? 2 : 4;
+  const Range rx = range_of(mixed_qkv, T * C * esz), rw = range_of(weight, C * K * 4);
+  const Range rb = bias ? range_of(bias, C * 4) : Range{0, 0};
+  const Range rsi = conv_state_in ? range_of(conv_state_in, N * C * K * esz) : Range{0, 0};
+  const Range rcu = cu_seqlens ? range_of(cu_seqlens, (N + 1) * 4) : Range{0, 0};
+  const size_t qkb = T * a.nqk * a.dk * esz;
+  const Range rq = range_of(q, qkb), rk = range_of(k, qkb), rv = range_of(v, T * a.nv * a.dv * esz);
+  const Range rso = conv_state_out ? range_of(conv_state_out, N * C * K * esz) : Range{0, 0};
+  for (Range o : {rq, rk, rv, rso})
+    for (Range i : {rx, rw, rb, rcu})
+      if (overlap(o, i)) return GDN_ERR_ALIAS;
+  if (overlap(rq, rk) || overlap(rq, rv) || overlap(rk, rv) || overlap(rso, rq) || overlap(rso, rk) ||
+      overlap(rso, rv))
+    return GDN_ERR_ALIAS;
+  for (Range o : {rq, rk, rv})
+    if (overlap(o, rsi)) return GDN_ERR_ALIAS;
+  if (conv_state_out && conv_state_in && conv_state_out != conv_state_in && overlap(rso, rsi))
+    return GDN_ERR_ALIAS;
+  rc = check_device();
+  if (rc) return rc;
+  a.state_in = conv_state_in; a.state_out = conv_state_out; a.cu = cu_seqlens;
+  a.uniform_len = cu_seqlens ? 0 : (int32_t)(total_tokens / num_seqs);
+  a.total_tokens = total_tokens;
+  const cudaError_t e = gdn::launch_conv_fwd(a, p->io_dtype == GDN_DTYPE_BF16, static_cast<cudaStream_t>(cuda_stream));
+  return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+GDN_API int gdn_qkv_conv_update(const void* mixed_qkv, const float* weight, const float* bias, void* conv_state,
+                                const int32_t* slot_ids, int32_t num_slots, int32_t num_seqs,
+                                int32_t kernel_size, void* q, void* k, void* v, const gdn_params_t* p,
+                                void* cuda_stream) {
+  gdn::ConvArgs a;
+  int rc = conv_common(mixed_qkv, weight, bias, kernel_size, q, k, v, num_seqs, p, a);
+  if (rc) return rc;
+  if (!conv_state) return GDN_ERR_NULL;
+  if (!aligned16(conv_state)) return GDN_ERR_ALIGN;
+  if (slot_ids) {
+    if (num_slots < 1) return GDN_ERR_SHAPE;
+    if (!aligned4(slot_ids)) return GDN_ERR_ALIGN;
+  }
+  const size_t N = (size_t)num_seqs, C = (size_t)a.channels, K = kernel_size;
+  const size_t esz = p->io_dtype == GDN_DTYPE_BF16 ? 2 : 4;
+  const size_t rows = slot_ids ? (size_t)num_slots : N;
+  const Range rx = range_of(mixed_qkv, N * C * esz), rw = range_of(weight, C * K * 4);
+  const Range rb = bias ? range_of(bias, C * 4) : Range{0, 0};
+  const Range rsl = slot_ids ? range_of(slot_ids, N * 4) : Range{0, 0};
+  const Range rs = range_of(conv_state, rows * C * K * esz);
+  const size_t qkb = N * a.nqk * a.dk * esz;
+  const Range rq = range_of(q, qkb), rk = range_of(k, qkb), rv = range_of(v, N * a.nv * a.dv * esz);
+  for (Range o : {rq, rk, rv, rs})
+    for (Range i : {rx, rw, rb, rsl})
+      if (overlap(o, i)) return GDN_ERR_ALIAS;
+  if (overlap(rq, rk) || overlap(rq, rv) || overlap(rk, rv) || overlap(rs, rq) || overlap(rs, rk) ||
+      overlap(rs, rv))
+    return GDN_ERR_ALIAS;
+  rc = check_device();
+  if (rc) return rc;
+  a.state_in = conv_state; a.state_out = conv_state; a.slots = slot_ids; a.num_slots = num_slots;
+  a.total_tokens = num_seqs;
+  const cudaError_t e =
+      gdn::launch_conv_update(a, p->io_dtype == GDN_DTYPE_BF16, static_cast<cudaStream_t>(cuda_stream));
   return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

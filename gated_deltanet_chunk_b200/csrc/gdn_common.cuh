@@ -55,6 +55,31 @@ struct StepArgs {
   const void* nz;      // [N, Nv, Dv] gate of the RMSNorm epilogue, or nullptr (no norm)
   const float* nw;     // [Dv] RMSNorm gain (with nz)
   float neps;          // RMSNorm eps (with nz)
+  const void* cx;      // [N, C] packed q|k|v projection when the conv is fused (q, k, v unused), or nullptr
+  void* cstate;        // [rows, C, cks] conv state (rows as the recurrent state), updated in place
+  const float* cw;     // [C, cks] conv taps
+  const float* cb;     // [C] conv bias or nullptr
+  int32_t cks;         // conv taps, 1..4
+};
+
+// Arguments of the causal conv1d + SiLU of the packed q|k|v channels.
+struct ConvArgs {
+  const void* x;             // [T, channels] (prefill) or [N, channels] (decode), io dtype
+  const float* weight;       // [channels, ksize]
+  const float* bias;         // [channels] or nullptr
+  const void* state_in;      // [N, channels, ksize] window before each sequence, or nullptr (zeros)
+  void* state_out;           // [N, channels, ksize] (prefill: or nullptr); decode: the state, in place
+  const int32_t* cu;         // [N + 1] or nullptr (equal lengths)
+  const int32_t* slots;      // decode: [N] state row of each sequence, or nullptr (row n)
+  int32_t num_slots;
+  int32_t uniform_len;       // sequence length when cu == nullptr
+  int32_t num_seqs;
+  int64_t total_tokens;
+  int32_t channels, ksize;   // channels = 2 nqk dk + nv dv
+  int32_t nqk, nv, dk, dv;
+  void* q;                   // [T or N, nqk, dk] outputs
+  void* k;
+  void* v;                   // [T or N, nv, dv]
 };
 
 template <typename T> __device__ __forceinline__ float to_f32(T x);

@@ -23,4 +23,9 @@ cudaError_t launch_recurrent_step(const StepArgs& a, int dk, int dv, int io_bf16
 cudaError_t launch_gated_rmsnorm(const void* o, const void* z, const float* w, float eps, void* y,
                                  int64_t rows, int dim, int io_bf16, cudaStream_t s);
 
+// Causal depthwise conv1d + SiLU of q|k|v: prefill (with the final conv_state
+// when state_out is set) and the one-token decode update; ksize in [1, 4].
+cudaError_t launch_conv_fwd(const ConvArgs& a, int io_bf16, cudaStream_t s);
+cudaError_t launch_conv_update(const ConvArgs& a, int io_bf16, cudaStream_t s);
+
 }  // namespace gdn

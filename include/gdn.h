@@ -215,6 +215,18 @@ int gdn_recurrent_step_gated(const void *q, const void *k, const void *v,
  *                    inputs for the overlap rules; norm_eps is finite and >= 0
  *                    (the layer's default is 1e-6).  A padding slot's decode row
  *                    stays zero.
+ *   conv_x,          causal conv fused ahead of the decode step (gdn_recurrent_step_ex
+ *   conv_state,      only): non-NULL conv_x => q, k, v must be NULL and the step
+ *   conv_weight,     forms them in-kernel from the packed projection, exactly as
+ *   conv_bias,       gdn_qkv_conv_update would (without rounding them to io_dtype):
+ *   conv_kernel_size   conv_x      [N, C] io_dtype, C = 2 Nqk Dk + Nv Dv, 16-byte aligned
+ *                      conv_state  [N, C, K] io_dtype (rows as the recurrent state:
+ *                                  with slot_ids, [num_slots, C, K] and the same
+ *                                  slots), 16-byte aligned, updated in place
+ *                      conv_weight [C, K] fp32;  conv_bias [C] fp32 or NULL
+ *                      conv_kernel_size K in [1, 4]
+ *                    The Nv / Nqk v-heads of a qk-head run as one thread-block
+ *                    cluster, so Nv / Nqk must be at most 8 (else GDN_ERR_SHAPE).
  */
 typedef struct {
     const float *A_log;
@@ -224,15 +236,22 @@ typedef struct {
     const void *norm_z;
     const float *norm_weight;
     float norm_eps;
+    const void *conv_x;
+    void *conv_state;
+    const float *conv_weight;
+    const float *conv_bias;
+    int32_t conv_kernel_size;
 } gdn_ext_t;
 
 /*
  * gdn_chunk_fwd_ex / gdn_recurrent_step_ex -- gdn_chunk_fwd / gdn_recurrent_step
  * with the fusions selected in `ext` (any combination).  Every argument, shape
  * rule, overlap rule and status code of the plain calls applies; `ext` adds its
- * own (GDN_ERR_NULL for a half-given gate or a norm_z without norm_weight,
- * GDN_ERR_SHAPE for num_slots < 1 or a bad norm_eps, GDN_ERR_ALIGN, GDN_ERR_ALIAS
- * when out overlaps norm_z or norm_weight).
+ * own (GDN_ERR_NULL for a half-given gate, a norm_z without norm_weight or a
+ * conv_x without conv_state / conv_weight; GDN_ERR_SHAPE for num_slots < 1, a
+ * bad norm_eps or conv_kernel_size, q / k / v given together with conv_x, or
+ * conv_x on gdn_chunk_fwd_ex, whose prefill conv is gdn_qkv_conv_fwd;
+ * GDN_ERR_ALIGN; GDN_ERR_ALIAS when an output overlaps any of these inputs).
  */
 int gdn_chunk_fwd_ex(const void *q, const void *k, const void *v,
                      const float *g, const float *beta,
@@ -262,6 +281,55 @@ int gdn_recurrent_step_ex(const void *q, const void *k, const void *v,
 int gdn_gated_rmsnorm(const void *o, const void *z, const float *weight, float eps,
                       void *y, int64_t rows, int32_t dim, int32_t io_dtype,
                       void *cuda_stream);
+
+/*
+ * gdn_qkv_conv_fwd / gdn_qkv_conv_update -- the causal depthwise conv1d + SiLU
+ * that turns the layer's packed projection mixed_qkv = [q | k | v] into the
+ * q, k, v of the calls above (walkthrough section 一(一)3, qkv 卷积部分; the
+ * decode form is its torch_causal_conv1d_update).  With C = 2 Nqk Dk + Nv Dv
+ * channels (shapes and io_dtype from p; p's qk_l2norm, scale and kernel are not
+ * used) and K = kernel_size taps:
+ *
+ *   y[t, c] = silu(bias[c] + sum_{i < K} weight[c, i] * in(t - (K - 1) + i))
+ *
+ * where in(p) is the sequence's input at position p, or for p < 0 the window
+ * cached before it, conv_state[n, c, K + p] (zeros when no state is given).
+ * Channel c < Nqk Dk is stored to q[t, c], c < 2 Nqk Dk to k[t, c - Nqk Dk], the
+ * rest to v[t, c - 2 Nqk Dk]; q, k are [rows, Nqk, Dk] and v [rows, Nv, Dv] in
+ * io_dtype, as gdn_chunk_fwd / gdn_recurrent_step read them.  A conv_state row
+ * is [C, K] in io_dtype holding the last K inputs (pre-convolution), the
+ * newest at index K - 1.  All arithmetic is fp32; silu(x) = x / (1 + exp(-x)).
+ *
+ *   mixed_qkv   [T, C] (prefill, packed sequences) or [N, C] (decode), io_dtype
+ *   weight      [C, K] fp32;  bias [C] fp32 or NULL (4-byte aligned)
+ *   kernel_size K in [1, 4]
+ *
+ * gdn_qkv_conv_fwd (prefill over N sequences, cu_seqlens as in gdn_chunk_fwd):
+ *   conv_state_in   [N, C, K] or NULL (each sequence starts after zeros)
+ *   conv_state_out  [N, C, K] or NULL: the last K inputs of [window, sequence]
+ *                   (zero filled on the left when fewer exist); may be
+ *                   conv_state_in (updated in place), may not overlap it otherwise
+ * gdn_qkv_conv_update (one token per sequence):
+ *   conv_state      [N, C, K] (or [num_slots, C, K] with slot_ids), updated in
+ *                   place: shifted by one, the new input at index K - 1
+ *   slot_ids        [N] int32 or NULL, as gdn_recurrent_step_slots: an id
+ *                   outside [0, num_slots) is a padding sequence (zero q, k, v;
+ *                   no state touched)
+ *
+ * q, k, v and the output state may not overlap the inputs or each other.
+ * Status codes as for gdn_chunk_fwd.
+ */
+int gdn_qkv_conv_fwd(const void *mixed_qkv, const float *weight, const float *bias,
+                     const void *conv_state_in, const int32_t *cu_seqlens,
+                     int32_t num_seqs, int64_t total_tokens, int32_t kernel_size,
+                     void *q, void *k, void *v, void *conv_state_out,
+                     const gdn_params_t *p, void *cuda_stream);
+
+int gdn_qkv_conv_update(const void *mixed_qkv, const float *weight, const float *bias,
+                        void *conv_state, const int32_t *slot_ids, int32_t num_slots,
+                        int32_t num_seqs, int32_t kernel_size,
+                        void *q, void *k, void *v,
+                        const gdn_params_t *p, void *cuda_stream);
 
 /*
  * gdn_device_status -- synchronise `cuda_stream`, then read and clear the

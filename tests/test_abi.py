@@ -213,3 +213,65 @@ def test_gated_rmsnorm_validation(L):
     if not torch.cuda.is_available():
         assert call(y=O) in (-5, -6)          # in place is valid: stops at the device check
         assert call() in (-5, -6)
+
+
+def test_conv_validation(L):
+    import torch
+    vp = ctypes.c_void_p
+    p = _p(nqk=2, nv=4, dk=128, dv=128)                 # C = 1024
+    X, Wt, Q, K_, V = A, A + 0x1000000, A + 0x2000000, A + 0x3000000, A + 0x4000000
+
+    def fwd(x=X, w=Wt, b=None, si=None, cu=None, n=2, T=256, ks=4, q=Q, k=K_, v=V, so=None, pp=p):
+        return L.gdn_qkv_conv_fwd(vp(x), vp(w), vp(b), vp(si), vp(cu), n, T, ks, vp(q), vp(k), vp(v), vp(so),
+                                  ctypes.byref(pp), None)
+    assert fwd(x=None) == -1
+    assert fwd(q=None) == -1
+    assert fwd(ks=0) == -2 and fwd(ks=5) == -2          # taps in [1, 4]
+    assert fwd(T=255) == -2                             # uneven split without cu_seqlens
+    assert fwd(pp=_p(nqk=3, nv=4)) == -2
+    assert fwd(x=X + 8) == -3
+    assert fwd(w=Wt + 2) == -3
+    assert fwd(q=X) == -4                               # q over the input
+    assert fwd(k=Q + 4096) == -4                        # k over q
+    assert fwd(si=A + 0x5000000, so=A + 0x5000000 + 64) == -4   # partial state overlap
+    assert fwd(so=Wt) == -4                             # state over the weight
+
+    def upd(st=A + 0x5000000, slots=None, ns=0, q=Q):
+        return L.gdn_qkv_conv_update(vp(X), vp(Wt), None, vp(st), vp(slots), ns, 4, 4, vp(q), vp(K_), vp(V),
+                                     ctypes.byref(p), None)
+    assert upd(st=None) == -1
+    assert upd(slots=A + 0x6000000, ns=0) == -2
+    assert upd(slots=A + 0x6000002, ns=8) == -3
+    assert upd(q=A + 0x5000000) == -4                   # q over the state
+    if not torch.cuda.is_available():
+        assert fwd() in (-5, -6)
+        assert fwd(si=A + 0x5000000, so=A + 0x5000000) in (-5, -6)   # in place is valid
+        assert upd() in (-5, -6)
+
+
+def test_ext_conv_validation(L):
+    import gated_deltanet_chunk_b200 as g
+    import torch
+    vp = ctypes.c_void_p
+    CX, CS, CW = A + 0xC000000, A + 0xD000000, A + 0xE000000
+
+    def step(q=None, pp=None, **kw):
+        x = g.GdnExt(conv_x=CX, conv_state=CS, conv_weight=CW, conv_kernel_size=4)
+        for k_, v_ in kw.items():
+            setattr(x, k_, v_)
+        pp = pp or _p()
+        return L.gdn_recurrent_step_ex(vp(q), None, None, vp(A + 0x300000), vp(A + 0x400000), vp(A + 0x500000),
+                                       vp(A + 0x900000), 4, ctypes.byref(pp), ctypes.byref(x), None)
+    assert step(q=A) == -2                                     # q given with the fused conv
+    assert step(conv_state=None) == -1
+    assert step(conv_kernel_size=5) == -2
+    assert step(pp=_p(nqk=1, nv=16)) == -2                     # group of 16 v-heads: no cluster that large
+    assert step(conv_x=CX + 8) == -3
+    assert step(conv_state=A + 0x500000) == -4                 # conv state over the recurrent state
+    assert step(conv_x=A + 0x900000) == -4                     # out over the projection
+    x = g.GdnExt(conv_x=CX, conv_state=CS, conv_weight=CW, conv_kernel_size=4)
+    assert L.gdn_chunk_fwd_ex(vp(A), vp(A + 0x1000000), vp(A + 0x2000000), vp(A + 0x3000000), vp(A + 0x4000000),
+                              None, None, 2, 256, 64, vp(A + 0x5000000), None, ctypes.byref(_p()),
+                              ctypes.byref(x), None) == -2         # no fused conv on the chunked call
+    if not torch.cuda.is_available():
+        assert step() in (-5, -6)

@@ -195,3 +195,25 @@ def make_norm_inputs(shape, io: str = "bf16", seed: int = 0, device: str = "cpu"
     z = torch.randn(*shape, generator=gen, device=device).to(dtype).contiguous()
     w = (torch.rand(shape[-1], generator=gen, device=device) + 0.5).contiguous()
     return z, w
+
+
+def make_conv_inputs(rows: int, nqk: int, nv: int, dk: int, dv: int, ksize: int = 4, io: str = "bf16",
+                     seed: int = 0, num_states: int = 0, bias: bool = True, device: str = "cpu"):
+    """Inputs of the causal conv1d + SiLU over packed [q | k | v] channels.
+
+    mixed_qkv [rows, C] ~ N(0, 1) (the layer's projection of unit-scale hidden
+    states), C = 2 nqk dk + nv dv; weight [C, K] ~ U(-1/sqrt(K), 1/sqrt(K)) and
+    bias [C] likewise (torch's default Conv1d init for a depthwise conv, fan-in
+    K); conv states [num_states, C, K] ~ N(0, 1) in the io dtype (cached
+    pre-convolution inputs), or None.
+    """
+    gen = torch.Generator(device=device).manual_seed(int(seed) + 104729)
+    dtype = torch.float32 if io == "f32" else torch.bfloat16
+    C = 2 * nqk * dk + nv * dv
+    bound = 1.0 / float(ksize) ** 0.5
+    x = torch.randn(rows, C, generator=gen, device=device).to(dtype).contiguous()
+    w = ((torch.rand(C, ksize, generator=gen, device=device) * 2 - 1) * bound).contiguous()
+    b = ((torch.rand(C, generator=gen, device=device) * 2 - 1) * bound).contiguous() if bias else None
+    st = (torch.randn(num_states, C, ksize, generator=gen, device=device).to(dtype).contiguous()
+          if num_states else None)
+    return dict(x=x, weight=w, bias=b, state=st, C=C)
