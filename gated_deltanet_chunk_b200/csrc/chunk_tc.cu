@@ -396,89 +396,117 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ok = !named_bar_any(1, 256, *abort_flag != 0);  // also: A^T is in M
       if (!ok) break;
-      // T = (I - A)^-1 over 32 x 32 blocks, in fp32 on the CUDA cores
-      // (A is strictly lower triangular, so T is unit lower triangular):
-      //   T11 = (I - A11)^-1, T22 = (I - A22)^-1: one column per lane (warps 0, 1),
-      //     from T = I + A T top to bottom; each replaces A^T in its block of M
-      //   Y = A21 T11 into M's block (1,0), then T21 = T22 Y over A21^T in block (0,1)
-      if (warp < 2) {
-        const int w = warp;
-        float* mb = ms + 32 * w * MS_LD + 32 * w;  // block (w, w); row k = column k of A_ww
-        float x[32];
+      // T = (I - A)^-1 in fp32 on the CUDA cores, by blocks (A is strictly lower
+      // triangular, T unit lower triangular).  M holds A^T on entry; each T block
+      // is written over an A^T block that is no longer needed, ending with T11,
+      // T22 row-major in M's diagonal 32 x 32 blocks and T21 in block (0, 1).
+      //   1. the four 16 x 16 diagonal blocks, T = I + A T from the top, one per
+      //      warp (0, 1, 4, 5; one column per lane); meanwhile warps 2, 3, 6, 7
+      //      store P, whose rows they hold
+      //   2. both 32 x 32 diagonal blocks: T_10 = T_11 (A_10 T_00) on 16 x 16 blocks
+      //   3. T21 = T22 (A21 T11) on 32 x 32 blocks, all 8 warps, 2 x 2 tiles
+      if (krow) {
+        const int b = (warp & 1) | ((warp >> 2) << 1);  // warps 0, 1, 4, 5 -> blocks 0..3
+        float* mb = ms + 16 * b * MS_LD + 16 * b;       // row k of this block of M = column k of A_bb
+        if (lane < 16) {
+          float x[16];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) x[i] = (i == lane) ? 1.f : 0.f;
-        // column k of A_ww (rows > k) is loaded one step ahead of its use
-        float4 cur[8], nxt[8];
+          for (int i = 0; i < 16; ++i) x[i] = (i == lane) ? 1.f : 0.f;
+          float4 cur[4], nxt[4];
 #pragma unroll
-        for (int v = 0; v < 8; ++v) cur[v] = *reinterpret_cast<const float4*>(mb + 4 * v);
+          for (int v = 0; v < 4; ++v) cur[v] = *reinterpret_cast<const float4*>(mb + 4 * v);
 #pragma unroll
-        for (int k = 0; k < 31; ++k) {
-          if (k + 1 < 31) {
+          for (int k = 0; k < 15; ++k) {
+            if (k + 1 < 15) {
 #pragma unroll
-            for (int v = (k + 2) >> 2; v < 8; ++v)
-              nxt[v] = *reinterpret_cast<const float4*>(mb + (k + 1) * MS_LD + 4 * v);
+              for (int v = (k + 2) >> 2; v < 4; ++v)
+                nxt[v] = *reinterpret_cast<const float4*>(mb + (k + 1) * MS_LD + 4 * v);
+            }
+#pragma unroll
+            for (int i = k + 1; i < 16; ++i) {
+              const float4 y = cur[i >> 2];
+              const float aik = (i & 3) == 0 ? y.x : (i & 3) == 1 ? y.y : (i & 3) == 2 ? y.z : y.w;
+              x[i] = fmaf(aik, x[k], x[i]);
+            }
+#pragma unroll
+            for (int v = 0; v < 4; ++v) cur[v] = nxt[v];
           }
+          __syncwarp(0x0000ffffu);
 #pragma unroll
-          for (int i = k + 1; i < 32; ++i) {
-            const float4 y = cur[i >> 2];
-            const float aik = (i & 3) == 0 ? y.x : (i & 3) == 1 ? y.y : (i & 3) == 2 ? y.z : y.w;
-            x[i] = fmaf(aik, x[k], x[i]);
-          }
-#pragma unroll
-          for (int v = 0; v < 8; ++v) cur[v] = nxt[v];
+          for (int i = 0; i < 16; ++i) mb[i * MS_LD + lane] = x[i];  // T_bb, row-major
         }
-        __syncwarp();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) mb[i * MS_LD + lane] = x[i];  // T_ww, row-major
+      } else {
+        ptx::st_half_packed(ps + PS_P, r, hf, pk0);  // P
+        ptx::fence_proxy_async_smem();
+        ptx::st_half_packed_remote(rpa + PS_P, rbar, r, hf, pk0);
       }
       named_bar_n(1, 256);
-      // Y = A21 T11 and T21 = T22 Y on warps 0-3 (one per scheduler): each of
-      // 128 threads owns a 2 x 4 output tile
-      const int i2 = 2 * (t >> 3), j4 = 4 * (t & 7);
-      if (warp < 4) {
-        // Y[i][j] = sum_k A21[i][k] T11[k][j] = sum_k M[k][32 + i] M[k][j]
-        float y[2][4] = {};
+      {
+        // 2. pair p (blocks 2p, 2p + 1): thread -> row i, columns j0, j0 + 1 of a 16 x 16 block
+        const int pr = t >> 7, idx = t & 127, i = idx >> 3, j0 = 2 * (idx & 7);
+        float* base = ms + 32 * pr * MS_LD + 32 * pr;
+        // Y = A_10 T_00:  A_10[i][k] = base[k][16 + i] (A^T),  T_00[k][j] = base[k][j]
+        float y0 = 0.f, y1 = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const float a10 = base[k * MS_LD + 16 + i];
+          const float2 t00 = *reinterpret_cast<const float2*>(base + k * MS_LD + j0);
+          y0 = fmaf(a10, t00.x, y0);
+          y1 = fmaf(a10, t00.y, y1);
+        }
+        *reinterpret_cast<float2*>(base + (16 + i) * MS_LD + j0) = make_float2(y0, y1);  // over A^T's zero block
+        named_bar_n(1, 256);
+        // T_10 = T_11 Y:  T_11[i][k] = base[16 + i][16 + k],  Y[k][j] = base[16 + k][j]
+        float z0 = 0.f, z1 = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const float t11 = base[(16 + i) * MS_LD + 16 + k];
+          const float2 yk = *reinterpret_cast<const float2*>(base + (16 + k) * MS_LD + j0);
+          z0 = fmaf(t11, yk.x, z0);
+          z1 = fmaf(t11, yk.y, z1);
+        }
+        named_bar_n(1, 256);  // every read of Y is done
+        *reinterpret_cast<float2*>(base + (16 + i) * MS_LD + j0) = make_float2(z0, z1);
+        // the upper right 16 x 16 of the 32 x 32 block (A_10^T, consumed) becomes T's zeros
+        *reinterpret_cast<float2*>(base + i * MS_LD + 16 + j0) = make_float2(0.f, 0.f);
+      }
+      named_bar_n(1, 256);
+      {
+        // 3. 32 x 32 blocks: thread -> rows i2, i2 + 1 and columns j2, j2 + 1
+        const int i2 = 2 * (t >> 4), j2 = 2 * (t & 15);
+        // Y = A21 T11:  A21[i][k] = M[k][32 + i],  T11[k][j] = M[k][j]
+        float y[2][2] = {};
 #pragma unroll
         for (int k = 0; k < 32; ++k) {
           const float2 a = *reinterpret_cast<const float2*>(ms + k * MS_LD + 32 + i2);
-          const float4 b = *reinterpret_cast<const float4*>(ms + k * MS_LD + j4);
-          const float av2[2] = {a.x, a.y}, bv4[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-          for (int r2 = 0; r2 < 2; ++r2)
-#pragma unroll
-            for (int c2 = 0; c2 < 4; ++c2) y[r2][c2] = fmaf(av2[r2], bv4[c2], y[r2][c2]);
+          const float2 b = *reinterpret_cast<const float2*>(ms + k * MS_LD + j2);
+          y[0][0] = fmaf(a.x, b.x, y[0][0]); y[0][1] = fmaf(a.x, b.y, y[0][1]);
+          y[1][0] = fmaf(a.y, b.x, y[1][0]); y[1][1] = fmaf(a.y, b.y, y[1][1]);
         }
 #pragma unroll
         for (int r2 = 0; r2 < 2; ++r2)
-          *reinterpret_cast<float4*>(ms + (32 + i2 + r2) * MS_LD + j4) = make_float4(y[r2][0], y[r2][1], y[r2][2], y[r2][3]);
-      }
-      named_bar_n(1, 256);
-      if (warp < 4) {
-        // T21[i][j] = sum_k T22[i][k] Y[k][j] = sum_k M[32 + i][32 + k] M[32 + k][j]
-        float y[2][4] = {};
+          *reinterpret_cast<float2*>(ms + (32 + i2 + r2) * MS_LD + j2) = make_float2(y[r2][0], y[r2][1]);
+        named_bar_n(1, 256);
+        // T21 = T22 Y:  T22[i][k] = M[32 + i][32 + k],  Y[k][j] = M[32 + k][j]; into block (0, 1)
+        float z[2][2] = {};
 #pragma unroll
         for (int k4 = 0; k4 < 32; k4 += 4) {
-          float a[2][4], b[4][4];
-#pragma unroll
-          for (int r2 = 0; r2 < 2; ++r2) {
-            const float4 v = *reinterpret_cast<const float4*>(ms + (32 + i2 + r2) * MS_LD + 32 + k4);
-            a[r2][0] = v.x; a[r2][1] = v.y; a[r2][2] = v.z; a[r2][3] = v.w;
-          }
+          const float4 a0 = *reinterpret_cast<const float4*>(ms + (32 + i2) * MS_LD + 32 + k4);
+          const float4 a1 = *reinterpret_cast<const float4*>(ms + (32 + i2 + 1) * MS_LD + 32 + k4);
+          const float av[2][4] = {{a0.x, a0.y, a0.z, a0.w}, {a1.x, a1.y, a1.z, a1.w}};
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const float4 v = *reinterpret_cast<const float4*>(ms + (32 + k4 + kk) * MS_LD + j4);
-            b[kk][0] = v.x; b[kk][1] = v.y; b[kk][2] = v.z; b[kk][3] = v.w;
+            const float2 b = *reinterpret_cast<const float2*>(ms + (32 + k4 + kk) * MS_LD + j2);
+#pragma unroll
+            for (int r2 = 0; r2 < 2; ++r2) {
+              z[r2][0] = fmaf(av[r2][kk], b.x, z[r2][0]);
+              z[r2][1] = fmaf(av[r2][kk], b.y, z[r2][1]);
+            }
           }
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-#pragma unroll
-            for (int r2 = 0; r2 < 2; ++r2)
-#pragma unroll
-              for (int c2 = 0; c2 < 4; ++c2) y[r2][c2] = fmaf(a[r2][kk], b[kk][c2], y[r2][c2]);
         }
 #pragma unroll
         for (int r2 = 0; r2 < 2; ++r2)
-          *reinterpret_cast<float4*>(ms + (i2 + r2) * MS_LD + 32 + j4) = make_float4(y[r2][0], y[r2][1], y[r2][2], y[r2][3]);
+          *reinterpret_cast<float2*>(ms + (i2 + r2) * MS_LD + 32 + j2) = make_float2(z[r2][0], z[r2][1]);
       }
       named_bar_n(1, 256);  // T21 is in M
       // products: stored locally first (and made visible to this CTA's tensor
@@ -488,11 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         spp[SP_SQ + t] = si[SI_SQ + t];
         if (t == 0) spp[SP_GAMMA] = si[SI_GAM];
       }
-      if (!krow) {
-        ptx::st_half_packed(ps + PS_P, r, hf, pk0);  // P
-        ptx::fence_proxy_async_smem();
-        ptx::st_half_packed_remote(rpa + PS_P, rbar, r, hf, pk0);
-      } else {
+      if (krow) {  // (P was stored while the diagonal blocks were solved)
         uint4 pk1[4];
         float x[32];  // row r of T, columns [c0, c0 + 32)
         if (r < 32 && hf == 1) {
