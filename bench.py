@@ -139,21 +139,28 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------- distributed
-def dist_setup(args):
+def dist_setup(args, backend="nccl"):
+    """One process per GPU: rank, world size and local rank from the launcher's
+    environment; a process group (NCCL over NVLink by default; gloo for the CPU
+    tests of this plumbing) when there is more than one rank."""
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return world, rank, local  # rank 0 alone runs the CPU oracle; no process group
+    if backend == "nccl":
+        torch.cuda.set_device(local if world > 1 else 0)
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    else:
-        torch.cuda.set_device(0)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     return world, rank, local
+
+
+def job_throughput(units_per_rank, world, steps, total_ms):
+    """Whole-job units/s: every rank's units over the slowest rank's time (weak scaling)."""
+    return units_per_rank * world * steps / (total_ms / 1e3)
 
 
 def barrier(world):
@@ -264,8 +271,7 @@ def run_ours(args, world, rank, local):
     per_launch_ms = [a.elapsed_time(b) for a, b in evs]
     kern_ms = statistics.mean(per_launch_ms)
     ms_per_step = total_ms / args.steps
-    tokens_all = T * world * args.steps
-    value = tokens_all / (total_ms / 1e3)
+    value = job_throughput(T, world, args.steps, total_ms)
 
     bytes_alg = prefill_bytes(T, nqk, nv, D, D, n, 2, s0=False, sf=True)
     fl_dense, fl_tri = prefill_flops(T // n, n, nv, C, D)
