@@ -392,10 +392,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ptx::mbar_wait_bounded(bars + BAR_PRODE + psl, par, kWaitNs)) *abort_flag = 1;
           if (!ptx::mbar_wait_cluster_bounded(bars + BAR_PEERF + psl, par, kWaitNs)) *abort_flag = 1;
         }
-        if (*abort_flag == 0) ptx::mbar_arrive_expect_tx_remote(rbar, kPushBytes);  // arm the other CTA's copy
       }
       ok = !named_bar_any(1, 256, *abort_flag != 0);  // also: A^T is in M
       if (!ok) break;
+      // arm the other CTA's copy, off the inverse's path (bytes that land first
+      // only drive the count below zero; the phase cannot complete before this
+      // arrival, and the previous phase completed before the slot was released)
+      if (t == 64) ptx::mbar_arrive_expect_tx_remote(rbar, kPushBytes);
       // T = (I - A)^-1 in fp32 on the CUDA cores, by blocks (A is strictly lower
       // triangular, T unit lower triangular).  M holds A^T on entry; each T block
       // is written over an A^T block that is no longer needed, ending with T11,
@@ -733,7 +736,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if ((c & 1) == (int)crank)
             ptx::mbar_arrive(bars + BAR_PRODE + psl);
           else
-            ptx::mbar_arrive_remote(ptx::mapa(ptx::smem_u32(bars + BAR_PEERF + psl), peer));
+            ptx::mbar_arrive_remote_relaxed(ptx::mapa(ptx::smem_u32(bars + BAR_PEERF + psl), peer));
         }
 #pragma unroll
         for (int qq = 0; qq < 4; ++qq) {
