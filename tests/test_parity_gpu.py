@@ -207,3 +207,28 @@ def test_tc_device_status_clean():
     w = W.make_prefill(num_seqs=1, seq_len=200, nqk=1, nv=2, d=128, io="bf16", seed=33)
     U.run_gpu_prefill(w, 64, kernel="tc")
     assert g.device_status() == 0
+
+
+# ---------------------------------------------------------------- maximum sequence count
+@pytest.mark.parametrize("io,d,kernel", [("bf16", 128, "tc"), ("f32", 64, "auto")])
+def test_max_num_seqs_prefill(io, d, kernel):
+    """65535 sequences (the ABI's limit: one grid dimension per sequence) of 0-3 tokens,
+    with initial states; every sequence checked against the oracle."""
+    lens = torch.randint(0, 4, (65535,), generator=torch.Generator().manual_seed(91))
+    w = W.make_prefill(lengths=lens, nqk=1, nv=1, d=d, io=io, init_state=True, seed=91)
+    _prefill_case(w, 64, kernel, "max-seqs-" + kernel)
+
+
+def test_max_num_seqs_decode():
+    """One decode step for 65535 sequences (grid y = sequences)."""
+    from gated_deltanet_chunk_b200 import recurrent_step
+    d = W.make_decode(num_seqs=65535, steps=1, nqk=1, nv=1, d=64, io="bf16", seed=92)
+    state = d["initial_state"].cuda()
+    out = recurrent_step(d["q"][0].cuda(), d["k"][0].cuda(), d["v"][0].cuda(), d["g"][0].cuda(),
+                         d["beta"][0].cuda(), state)
+    torch.cuda.synchronize()
+    import oracle
+    cu = torch.arange(65536, dtype=torch.int32)
+    ref_o, ref_s = oracle.recurrent(d["q"][0], d["k"][0], d["v"][0], d["g"][0], d["beta"][0],
+                                    d["initial_state"], cu)
+    U.check_prefill(out, state, ref_o, ref_s, cu, U.TOL["bf16"], "max-seqs-decode")
