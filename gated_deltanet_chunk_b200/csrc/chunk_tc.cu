@@ -17,9 +17,12 @@
 //     rounded to bf16, in shared memory as the B operand of the next
 //     chunk.  The critical path per chunk is three tensor-core round trips
 //     ([K;Q] S with U, then V', then D4) and three short epilogues; W itself
-//     is never formed.  The output rows (P V' + Q S) are finished by warps 10-11 while
-//     warps 8-9 start the next chunk.  The serial warps also refill this CTA's
-//     3-deep TMA ring of raw q/k/v tiles.
+//     is never formed.  P V' is issued by a second thread, so the thread that
+//     polls D4 goes straight from issuing it to waiting on it.  The output
+//     rows (P V' + Q S) are finished by warps 10-11 while warps 8-9 start the
+//     next chunk.  The serial warps also refill this CTA's 3-deep TMA ring of
+//     raw q/k/v tiles, and release each product slot (to the other CTA with a
+//     relaxed cluster arrive: it reports finished reads, nothing to publish).
 //
 // Algebra: the chunkwise form of the "手撕Qwen3-Next" walkthrough, section
 // 一(一)5(1), steps c-f, with the L2 norms folded into row scales
@@ -29,9 +32,11 @@
 //   G  = [K; Q] K^T                                     tcgen05 M=128 N=64 K=128
 //   A  = -strictLower(diag(beta rk) (K K^T) diag(rk) * Gamma)          CUDA cores
 //   P  = diag(rq) (Q K^T) diag(rk) * Gamma  (lower incl. diagonal)      CUDA cores
-//   T  = (I - A)^-1 over 32 x 32 blocks, fp32 in shared memory:     CUDA cores
-//        T11, T22 by forward substitution on T = I + A T (one column per lane),
-//        T21 = T22 (A21 T11) (two 32 x 32 products over 256 threads)
+//   T  = (I - A)^-1, fp32 in shared memory:                          CUDA cores
+//        the four 16 x 16 diagonal blocks by forward substitution on
+//        T = I + A T (one column per lane, one block per warp), then
+//        T_10 = T_11 (A_10 T_00) for both 32 x 32 blocks and
+//        T21 = T22 (A21 T11) for the whole, over all 256 intra threads
 //   serial:  U = T diag(beta) V,  [K S; Q S] = [K; Q] S                one round
 //            K S rounded to bf16                                      CUDA cores
 //            V' = U + (-T diag(beta exp(gcum) rk)) (K S) = U - W S      one round
