@@ -328,6 +328,25 @@ def run_ours(args, world, rank, local):
                                      "traffic": None, "peak_source": peak_src,
                                      "alg_bytes_per_launch": g_bytes}}
         del ga
+    # the varlen workload: 32 packed sequences of U[100, 16384] tokens with
+    # initial states (the configuration the parity tests sample by heads)
+    if not args.no_varlen:
+        wv = W.make_workload("varlen_bf16_nv32", seed=3 + rank, device=str(dev))
+        nvs, Tv = wv["num_seqs"], wv["T"]
+        ov = torch.empty(Tv, nv, D, dtype=torch.bfloat16, device=dev)
+        sv = torch.empty_like(wv["initial_state"])
+
+        def vstep():
+            gdn.chunk_fwd(wv["q"], wv["k"], wv["v"], wv["g"], wv["beta"], wv["initial_state"], wv["cu_seqlens"],
+                          chunk_size=C, out=ov, final_state=sv, kernel=args.kernel)
+
+        v_ms = time_steps(vstep, args.warmup, max(3, args.steps // 4), stream, world, dev)
+        vb = prefill_bytes(Tv, nqk, nv, D, D, nvs, 2, s0=True, sf=True)
+        res["varlen"] = hbm_line(v_ms, vb, peaks, peak_src, value=Tv * world / (v_ms / 1e3), unit="tokens/s",
+                                 workload="varlen_bf16_nv32", num_seqs=nvs, tokens=Tv,
+                                 call="gdn_chunk_fwd (cu_seqlens, initial and final state)",
+                                 gpu_launches=max(3, args.steps // 4))
+        del wv, ov, sv
     # the same workload with the gated RMSNorm epilogue fused into the output
     # stores (gdn_chunk_fwd_ex), and the epilogue on its own (gdn_gated_rmsnorm)
     if not args.no_norm:
@@ -636,6 +655,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-gated", action="store_true", help="skip the fused-gate prefill and decode lines")
     ap.add_argument("--no-slots", action="store_true", help="skip the slot-indexed decode line")
+    ap.add_argument("--no-varlen", action="store_true", help="skip the varlen prefill line")
     ap.add_argument("--no-conv", action="store_true",
                     help="skip the causal-conv lines (prefill conv, decode conv update)")
     ap.add_argument("--no-norm", action="store_true",

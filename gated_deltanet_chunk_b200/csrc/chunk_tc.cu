@@ -170,6 +170,30 @@ __device__ __forceinline__ bool named_bar_any(int id, int nthreads, bool flag) {
 }
 
 
+// The sequence this CTA runs: blockIdx.z is a rank, longest sequence first
+// (ties by index), so that with packed sequences of mixed lengths, which the
+// block scheduler starts in z order, the longest chains start earliest.  Each
+// thread ranks one sequence by comparing lengths; beyond kRankMax sequences
+// (or with equal lengths) the order is the identity.  Called by all threads.
+constexpr int kRankMax = 128;
+__device__ __forceinline__ int sequence_of_rank(const ChunkArgs& a, int rank, int* slot) {
+  if (a.cu == nullptr || a.num_seqs > kRankMax) return rank;
+  if (threadIdx.x == 0) *slot = rank;  // overwritten below; stays only if the ranks were inconsistent
+  __syncthreads();
+  const int i = threadIdx.x;
+  if (i < a.num_seqs) {
+    const int li = a.cu[i + 1] - a.cu[i];
+    int r = 0;
+    for (int q = 0; q < a.num_seqs; ++q) {
+      const int lq = a.cu[q + 1] - a.cu[q];
+      r += (lq > li) || (lq == li && q < i);
+    }
+    if (r == rank) *slot = i;
+  }
+  __syncthreads();
+  return *slot;
+}
+
 template <bool kRawGate>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -180,13 +204,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t raw_s = ptx::smem_u32(smem_raw);
   uint8_t* sm = smem_raw + (((raw_s + 1023u) & ~1023u) - raw_s);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int slice = blockIdx.x, h = blockIdx.y, n = blockIdx.z;
+  const int slice = blockIdx.x, h = blockIdx.y;
   const int j = h / (a.nv / a.nqk);
   const int nv = a.nv, dv = a.dv;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_BAR + NBAR * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_BAR + NBAR * 8 + 4);
+  int* seq_slot = reinterpret_cast<int*>(sm + OFF_BAR + NBAR * 8 + 8);
+  const int n = sequence_of_rank(a, (int)blockIdx.z, seq_slot);
   float* si = reinterpret_cast<float*>(sm + OFF_SCI);
   float* sp = reinterpret_cast<float*>(sm + OFF_SCP);
 
