@@ -2,7 +2,6 @@
 // kernel choice and launch on the caller's stream.  See include/gdn.h.
 #include <cmath>
 #include <cstdint>
-#include <mutex>
 
 #include "../../include/gdn.h"
 #include "gdn_common.cuh"

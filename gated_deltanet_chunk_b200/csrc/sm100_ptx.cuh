@@ -95,22 +95,10 @@ __device__ __forceinline__ uint32_t mapa(uint32_t saddr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
   return r;
 }
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint4 v) {
-  asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
-               "r"(v.w)
-               : "memory");
-}
-__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
-  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
-}
-// arrive on an mbarrier of another CTA of the cluster; orders this thread's prior
-// (and, cumulatively, observed) writes before it at cluster scope
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-// The same without release semantics: for an arrival that only reports that
-// reads are finished whose values the thread has already consumed (a release
-// arrive would also wait for this thread's earlier global stores).
+// Arrive on another CTA's mbarrier without release semantics: for an arrival
+// that only reports that reads are finished whose values the thread has
+// already consumed (a release arrive would also wait for this thread's earlier
+// global stores).
 __device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
@@ -155,7 +143,7 @@ __device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t cluster_ba
                "r"(bytes)
                : "memory");
 }
-__device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
+
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
@@ -338,29 +326,6 @@ __device__ __forceinline__ void st_half_packed_remote(uint32_t remote, uint32_t 
   for (int c = 0; c < 4; ++c) st_async_v4(remote + sw128_off(r, 4 * half + c), w[c], rbar);
 }
 
-// Like st_half_bf16 / st_row_bf16, also sending the same bytes with st.async
-// to `remote`, the shared::cluster address of the same tile in another CTA of
-// the cluster, completing transactions on that CTA's mbarrier `rbar`.
-__device__ __forceinline__ void st_half_bf16_dual(uint8_t* tile, uint32_t remote, uint32_t rbar, int r, int half,
-                                                  const float* v) {
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    const uint4 w = pack8_bf16(v + 8 * c);
-    const uint32_t off = sw128_off(r, 4 * half + c);
-    *reinterpret_cast<uint4*>(tile + off) = w;
-    st_async_v4(remote + off, w, rbar);
-  }
-}
-__device__ __forceinline__ void st_row_bf16_dual(uint8_t* tile, uint32_t remote, uint32_t rbar, int r,
-                                                 const float* v) {
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    const uint4 w = pack8_bf16(v + 8 * c);
-    const uint32_t off = sw128_off(r, c);
-    *reinterpret_cast<uint4*>(tile + off) = w;
-    st_async_v4(remote + off, w, rbar);
-  }
-}
 
 // Reads row r (64 bf16) of a swizzled tile into fp32.
 __device__ __forceinline__ void ld_row_bf16(const uint8_t* tile, int r, float* v) {
