@@ -102,6 +102,8 @@ def lib() -> ctypes.CDLL:
         L.gdn_qkv_conv_update.argtypes = [vp, fp, fp, vp, ip, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                           vp, vp, vp, ctypes.POINTER(GdnParams), vp]
         L.gdn_qkv_conv_update.restype = ctypes.c_int
+        L.gdn_selftest_wait_timeout.argtypes = [ctypes.c_int64, vp]
+        L.gdn_selftest_wait_timeout.restype = ctypes.c_int
         L.gdn_device_status.argtypes = [vp]
         L.gdn_device_status.restype = ctypes.c_int
         L.gdn_status_string.argtypes = [ctypes.c_int]
@@ -208,6 +210,12 @@ def recurrent_step_gated(q, k, v, a, b, A_log, dt_bias, state, out=None, qk_l2no
     """
     return _step_call("gdn_recurrent_step_gated", (a, b, A_log, dt_bias), q, k, v, state, out,
                       qk_l2norm, scale, stream, check)
+
+
+def selftest_wait_timeout(limit_us=2000, stream=None) -> int:
+    """Launch the failure-detection self-test (``gdn_selftest_wait_timeout``); then
+    ``device_status()`` reports GDN_ERR_DEVICE_TIMEOUT once."""
+    return lib().gdn_selftest_wait_timeout(int(limit_us), _stream(stream))
 
 
 def device_status(stream=None) -> int:

@@ -891,6 +891,24 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int64_t total_tokens, cudaStream
   return cudaGetLastError();
 }
 
+// Self-test of the failure detection: one CTA waits, with the same bounded
+// mbarrier wait the chunk kernel uses, on a barrier nothing arrives on; after
+// limit_ns it gives up and records the timeout in the status word.
+__global__ void selftest_wait_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&bar, 1);
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !ptx::mbar_wait_bounded(&bar, 0u, limit_ns)) atomicOr(&tc::g_status, 1u);
+}
+
+cudaError_t launch_selftest_wait(uint64_t limit_ns, cudaStream_t s) {
+  selftest_wait_kernel<<<1, 32, 0, s>>>(limit_ns);
+  return cudaGetLastError();
+}
+
 unsigned int chunk_tc_take_status() {
   unsigned int v = 0, zero = 0;
   if (cudaMemcpyFromSymbol(&v, tc::g_status, sizeof(v)) != cudaSuccess) return ~0u;

@@ -449,6 +449,14 @@ GDN_API int gdn_qkv_conv_update(const void* mixed_qkv, const float* weight, cons
   return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
+GDN_API int gdn_selftest_wait_timeout(int64_t limit_us, void* cuda_stream) {
+  if (limit_us < 1 || limit_us > 2000000) return GDN_ERR_SHAPE;
+  const int rc = check_device();
+  if (rc) return rc;
+  const cudaError_t e = gdn::launch_selftest_wait((uint64_t)limit_us * 1000u, static_cast<cudaStream_t>(cuda_stream));
+  return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
 GDN_API int gdn_device_status(void* cuda_stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(cuda_stream));
   if (e != cudaSuccess) return GDN_ERR_CUDA;

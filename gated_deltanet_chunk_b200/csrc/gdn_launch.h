@@ -15,6 +15,8 @@ bool chunk_tc_supported(int dk, int dv, int chunk, int io_bf16, int64_t total_to
 cudaError_t launch_chunk_tc(const ChunkArgs& a, int64_t total_tokens, cudaStream_t s);
 // Reads and clears the tensor-core kernel's device status word (bit 0: a bounded wait expired).
 unsigned int chunk_tc_take_status();
+// One CTA whose bounded wait on a barrier nothing arrives on expires after limit_ns.
+cudaError_t launch_selftest_wait(uint64_t limit_ns, cudaStream_t s);
 
 // One-token decode step; dk, dv in {64,128}.
 cudaError_t launch_recurrent_step(const StepArgs& a, int dk, int dv, int io_bf16, cudaStream_t s);

@@ -340,6 +340,16 @@ int gdn_qkv_conv_update(const void *mixed_qkv, const float *weight, const float 
  */
 int gdn_device_status(void *cuda_stream);
 
+/*
+ * gdn_selftest_wait_timeout -- self-test of the device-side failure detection.
+ * Launches one CTA on `cuda_stream` that waits, with the library's bounded
+ * mbarrier wait, on a barrier nothing arrives on; after limit_us microseconds
+ * (1 .. 2,000,000) the wait gives up and records the timeout in the status word
+ * that gdn_device_status reads, and the CTA returns.  Nothing faults or hangs,
+ * and the context stays usable.  Returns GDN_OK once launched.
+ */
+int gdn_selftest_wait_timeout(int64_t limit_us, void *cuda_stream);
+
 /* Human-readable name of a status code (static storage; never NULL). */
 const char *gdn_status_string(int status);
 

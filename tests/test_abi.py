@@ -275,3 +275,11 @@ def test_ext_conv_validation(L):
                               ctypes.byref(x), None) == -2         # no fused conv on the chunked call
     if not torch.cuda.is_available():
         assert step() in (-5, -6)
+
+
+def test_selftest_wait_timeout_validation(L):
+    import torch
+    assert L.gdn_selftest_wait_timeout(0, None) == -2
+    assert L.gdn_selftest_wait_timeout(2000001, None) == -2
+    if not torch.cuda.is_available():
+        assert L.gdn_selftest_wait_timeout(1000, None) in (-5, -6)
