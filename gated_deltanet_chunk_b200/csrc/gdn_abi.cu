@@ -114,7 +114,8 @@ static int chunk_fwd_impl(const void* q, const void* k, const void* v, const flo
                           const gdn_ext_t& x) {
   int rc = check_params(p);
   if (rc) return rc;
-  if (!q || !k || !v || !g || !beta || !out) return GDN_ERR_NULL;
+  // with no tokens nothing is read or written but the states: the token tensors may be NULL
+  if (total_tokens != 0 && (!q || !k || !v || !g || !beta || !out)) return GDN_ERR_NULL;
   rc = check_ext(x);
   if (rc) return rc;
   if (x.conv_x) return GDN_ERR_SHAPE;  // the prefill conv is gdn_qkv_conv_fwd
@@ -356,14 +357,15 @@ GDN_API int gdn_gated_rmsnorm(const void* o, const void* z, const float* weight,
 
 // Shared validation of the two conv calls; fills the launch block.
 static int conv_common(const void* x, const float* weight, const float* bias, int32_t kernel_size, void* q,
-                       void* k, void* v, int32_t num_seqs, const gdn_params_t* p, gdn::ConvArgs& a) {
+                       void* k, void* v, int32_t num_seqs, int64_t rows, const gdn_params_t* p, gdn::ConvArgs& a) {
   int rc = check_params(p);
   if (rc) return rc;
-  if (!x || !weight || !q || !k || !v) return GDN_ERR_NULL;
+  if (!weight) return GDN_ERR_NULL;
+  if (rows != 0 && (!x || !q || !k || !v)) return GDN_ERR_NULL;  // no rows: the tensors may be NULL
   if (kernel_size < 1 || kernel_size > 4) return GDN_ERR_SHAPE;
   if (num_seqs < 1 || num_seqs > 65535) return GDN_ERR_SHAPE;
   for (const void* ptr : {x, (const void*)q, (const void*)k, (const void*)v})
-    if (!aligned16(ptr)) return GDN_ERR_ALIGN;
+    if (ptr && !aligned16(ptr)) return GDN_ERR_ALIGN;
   if (!aligned4(weight) || (bias && !aligned4(bias))) return GDN_ERR_ALIGN;
   a = gdn::ConvArgs{};
   a.x = x; a.weight = weight; a.bias = bias; a.num_seqs = num_seqs; a.ksize = kernel_size;
@@ -378,9 +380,9 @@ GDN_API int gdn_qkv_conv_fwd(const void* mixed_qkv, const float* weight, const f
                              int64_t total_tokens, int32_t kernel_size, void* q, void* k, void* v,
                              void* conv_state_out, const gdn_params_t* p, void* cuda_stream) {
   gdn::ConvArgs a;
-  int rc = conv_common(mixed_qkv, weight, bias, kernel_size, q, k, v, num_seqs, p, a);
-  if (rc) return rc;
   if (total_tokens < 0 || total_tokens >= (int64_t(1) << 31)) return GDN_ERR_SHAPE;
+  int rc = conv_common(mixed_qkv, weight, bias, kernel_size, q, k, v, num_seqs, total_tokens, p, a);
+  if (rc) return rc;
   if (!cu_seqlens && total_tokens % num_seqs != 0) return GDN_ERR_SHAPE;
   for (const void* ptr : {conv_state_in, (const void*)conv_state_out, (const void*)cu_seqlens})
     if (ptr && !aligned16(ptr)) return GDN_ERR_ALIGN;
@@ -417,7 +419,7 @@ GDN_API int gdn_qkv_conv_update(const void* mixed_qkv, const float* weight, cons
                                 int32_t kernel_size, void* q, void* k, void* v, const gdn_params_t* p,
                                 void* cuda_stream) {
   gdn::ConvArgs a;
-  int rc = conv_common(mixed_qkv, weight, bias, kernel_size, q, k, v, num_seqs, p, a);
+  int rc = conv_common(mixed_qkv, weight, bias, kernel_size, q, k, v, num_seqs, num_seqs, p, a);
   if (rc) return rc;
   if (!conv_state) return GDN_ERR_NULL;
   if (!aligned16(conv_state)) return GDN_ERR_ALIGN;

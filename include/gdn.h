@@ -95,6 +95,8 @@ typedef struct {
  *   p              shapes and options (see gdn_params_t)
  *
  * Zero-length sequences are allowed: their final_state equals their initial state.
+ * With total_tokens = 0 the token tensors (q, k, v, g, beta, out) are not read or
+ * written and may be NULL; final_state then receives initial_state (or zeros).
  */
 int gdn_chunk_fwd(const void *q, const void *k, const void *v,
                   const float *g, const float *beta,
@@ -305,6 +307,7 @@ int gdn_gated_rmsnorm(const void *o, const void *z, const float *weight, float e
  *   kernel_size K in [1, 4]
  *
  * gdn_qkv_conv_fwd (prefill over N sequences, cu_seqlens as in gdn_chunk_fwd):
+ *   total_tokens    T >= 0; with T = 0, mixed_qkv, q, k and v may be NULL
  *   conv_state_in   [N, C, K] or NULL (each sequence starts after zeros)
  *   conv_state_out  [N, C, K] or NULL: the last K inputs of [window, sequence]
  *                   (zero filled on the left when fewer exist); may be

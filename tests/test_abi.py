@@ -283,3 +283,18 @@ def test_selftest_wait_timeout_validation(L):
     assert L.gdn_selftest_wait_timeout(2000001, None) == -2
     if not torch.cuda.is_available():
         assert L.gdn_selftest_wait_timeout(1000, None) in (-5, -6)
+
+
+def test_empty_batch_accepts_null_token_tensors(L):
+    import torch
+    vp = ctypes.c_void_p
+    p = _p()
+    S0, SF = A + 0x7000000, A + 0x8000000
+    rc = L.gdn_chunk_fwd(None, None, None, None, None, vp(S0), None, 2, 0, 64, None, vp(SF), ctypes.byref(p), None)
+    rc_tokens = L.gdn_chunk_fwd(None, None, None, None, None, vp(S0), None, 2, 256, 64, None, vp(SF),
+                                ctypes.byref(p), None)
+    assert rc_tokens == -1                        # with tokens the tensors are required
+    rc_conv = L.gdn_qkv_conv_fwd(None, vp(A), None, None, None, 2, 0, 4, None, None, None, vp(SF),
+                                 ctypes.byref(p), None)
+    if not torch.cuda.is_available():
+        assert rc in (-5, -6) and rc_conv in (-5, -6)   # valid: stops at the device check

@@ -226,3 +226,14 @@ def test_fused_conv_equals_two_launches_and_all_fusions():
         assert U.rel_inf(U.to_np(go[n]), ref_o[i]) <= U.TOL["bf16"], n
     assert U.rel_inf(U.to_np(s3), ref_s) <= U.TOL["bf16"]
     assert np.array_equal(U.to_np(cs3), ref_cs)
+
+
+def test_conv_fwd_empty_batch_keeps_the_windows():
+    """total_tokens = 0: no q, k, v rows; the new conv_state is the old window, bit for bit."""
+    from gated_deltanet_chunk_b200 import qkv_conv_fwd
+    c = W.make_conv_inputs(0, 2, 4, 64, 128, 4, "bf16", seed=97, num_states=3)
+    q, k, v, st = qkv_conv_fwd(c["x"].cuda(), c["weight"].cuda(), 2, 4, 64, 128, bias=c["bias"].cuda(),
+                               conv_state=c["state"].cuda(), cu_seqlens=torch.zeros(4, dtype=torch.int32).cuda())
+    torch.cuda.synchronize()
+    assert q.numel() == 0 and v.numel() == 0
+    assert torch.equal(st.cpu(), c["state"])
