@@ -77,7 +77,11 @@ typedef struct {
  *
  *   q, k           [T, Nqk, Dk]  io_dtype
  *   v              [T, Nv, Dv]   io_dtype
- *   g, beta        [T, Nv]       fp32   (g = log of the decay, beta = write strength)
+ *   g, beta        [T, Nv]       fp32   (g = log of the decay, beta = write strength).
+ *                  g <= 0 (a decay, as the layer's gate always is) where the
+ *                  tensor-core kernel runs: it splits the in-chunk decay into
+ *                  factors that are at most 1.  The CUDA-core kernel
+ *                  (GDN_KERNEL_SIMT) takes any finite g.
  *   initial_state  [N, Nv, Dk, Dv] fp32 (Dk rows, Dv contiguous) or NULL for zeros
  *   cu_seqlens     [N + 1] int32 device array: cu[0] = 0, non-decreasing, cu[N] = T;
  *                  sequence n owns tokens [cu[n], cu[n+1]) and starts from
