@@ -237,3 +237,36 @@ def test_conv_fwd_empty_batch_keeps_the_windows():
     torch.cuda.synchronize()
     assert q.numel() == 0 and v.numel() == 0
     assert torch.equal(st.cpu(), c["state"])
+
+
+def test_fused_conv_norm_decode_full_shape_sampled():
+    """The decode workload's shape (256 sequences, Nqk 16, Nv 32, D 128) with the conv and the
+    norm fused into the step, 3 steps; 8 sequences checked against the oracle (all heads)."""
+    from gated_deltanet_chunk_b200 import recurrent_step_ex
+    N, nqk, nv, steps = 256, 16, 32, 3
+    d = W.make_decode(num_seqs=N, steps=steps, nqk=nqk, nv=nv, io="bf16", seed=98)
+    c = W.make_conv_inputs(N * steps, nqk, nv, 128, 128, 4, "bf16", seed=98, num_states=N)
+    z, nw = W.make_norm_inputs(d["v"].shape, "bf16", seed=98)
+    x = c["x"].reshape(steps, N, c["C"]).cuda()
+    state, cst = d["initial_state"].cuda(), c["state"].cuda()
+    outs = []
+    for t in range(steps):
+        outs.append(recurrent_step_ex(None, None, None, d["g"][t].cuda(), d["beta"][t].cuda(), state,
+                                      norm_z=z[t].cuda(), norm_weight=nw.cuda(), conv_x=x[t], conv_state=cst,
+                                      conv_weight=c["weight"].cuda(), conv_bias=c["bias"].cuda(),
+                                      shapes=(nqk, nv, 128, 128)))
+    torch.cuda.synchronize()
+    pick_seqs = [0, 1, 37, 100, 128, 199, 254, 255]
+    idx = torch.as_tensor(pick_seqs)
+    xs = c["x"].reshape(steps, N, c["C"])[:, idx].transpose(0, 1).reshape(len(idx) * steps, c["C"])
+    cu = np.arange(len(idx) + 1, dtype=np.int32) * steps
+    y, ref_cs = oracle.causal_conv1d(xs, c["weight"], c["bias"], cu, c["state"][idx])
+    q, k, v = _split(y, nqk, nv, 128, 128)
+    pick = lambda t: t[:, idx].transpose(0, 1).reshape(len(idx) * steps, *t.shape[2:])
+    o, sf = oracle.recurrent(q, k, v, pick(d["g"]), pick(d["beta"]), d["initial_state"][idx], cu)
+    o = oracle.gated_rmsnorm(o, pick(z), nw, 1e-6).reshape(len(idx), steps, nv, 128)
+    go = torch.stack(outs, 1)[idx]
+    for i in range(len(idx)):
+        assert U.rel_inf(U.to_np(go[i]), o[i]) <= U.TOL["bf16"], pick_seqs[i]
+    assert U.rel_inf(U.to_np(state[idx.cuda()]), sf) <= U.TOL["bf16"]
+    assert np.array_equal(U.to_np(cst[idx.cuda()]), ref_cs)
