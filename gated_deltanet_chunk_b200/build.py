@@ -16,7 +16,7 @@ BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libgdn.so")
 
 SOURCES = ["gdn_abi.cu", "chunk_simt.cu", "chunk_tc.cu", "decode_step.cu", "gated_rmsnorm.cu", "causal_conv.cu"]
-HEADERS = ["gdn_common.cuh", "gdn_launch.h", "sm100_ptx.cuh"]
+HEADERS = ["gdn_common.cuh", "gdn_launch.h", "gdn_silu.cuh", "sm100_ptx.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

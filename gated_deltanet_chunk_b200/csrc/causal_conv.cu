@@ -15,9 +15,11 @@
 // The outputs go straight to the three tensors the chunk and decode kernels
 // read: channels [0, Nqk Dk) to q [T, Nqk, Dk], [Nqk Dk, 2 Nqk Dk) to k, the
 // rest to v [T, Nv, Dv].  Every kernel here is bound by HBM: x is read once
-// and q, k, v written once (the K - 1 earlier rows a thread re-reads are L1
-// hits).  A thread owns one 16-byte vector of channels (8 bf16 or 4 fp32).
+// and q, k, v written once (a prefill block also reads the K - 1 rows before
+// its first token, 3 in 128, which the neighbouring block has brought into
+// L2).  A thread owns one 16-byte vector of channels (8 bf16 or 4 fp32).
 #include "gdn_common.cuh"
+#include "gdn_silu.cuh"
 #include "gdn_launch.h"
 
 namespace gdn {
@@ -119,23 +121,48 @@ __device__ __forceinline__ int seq_of(const int32_t* cu, int num_seqs, int64_t t
 
 // Prefill: block (token block, channel block); thread = one channel vector over
 // kTokensPerBlock consecutive tokens, which may cross sequence boundaries.  The
-// K - 1 previous inputs stay in registers (a sliding window); the rows of the
-// next kBatch tokens are requested while the current kBatch are computed, so
-// loads stay in flight through the arithmetic (single-buffered batches of 8
-// measured 0.618 ms on the long prefill, this 0.495 ms).
-constexpr int kBatch = 4;
+// thread's input rows come through a ring of kDepth 16-byte cp.async copies in
+// shared memory, so kDepth - 1 rows stay in flight without holding registers.
+// A thread reads back only the slots it filled itself, so its own
+// cp.async.wait_group orders them and no block barrier is needed.  The K - 1
+// previous inputs stay in registers as a sliding window, and the token loop is
+// unrolled by 4 so that shifting it costs no moves.  On the long prefill
+// (65,536 tokens x 8192 channels, bf16) the steps measured: register-held
+// double buffer of 4 rows 0.494 ms; with the one-MUFU SiLU 0.406 ms; this ring
+// 0.381 ms; unrolled 0.358 ms.  Deeper rings (24) and three blocks per SM
+// (register spills) measured slower.
+constexpr int kDepth = 16;
+constexpr int kBlocksPerSM = 2;
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
 
 template <typename IO, int K>
-__global__ void __launch_bounds__(kThreads) conv_fwd_kernel(ConvArgs a) {
+__global__ void __launch_bounds__(kThreads, kBlocksPerSM) conv_fwd_kernel(ConvArgs a) {
   constexpr int E = V16<IO>::N;
+  extern __shared__ __align__(16) uint4 ring[];  // [kDepth][kThreads]
   const int c0 = (blockIdx.y * kThreads + threadIdx.x) * E;
   if (c0 >= a.channels) return;
   const int64_t t_begin = (int64_t)blockIdx.x * kTokensPerBlock;
   const int64_t t_end = min((int64_t)a.total_tokens, t_begin + kTokensPerBlock);
   if (t_begin >= t_end) return;
+  const IO* xc = static_cast<const IO*>(a.x) + c0;
+  const uint32_t rbase = (uint32_t)__cvta_generic_to_shared(ring + threadIdx.x);
+  // row tt into ring slot `slot`; one commit group per row (empty past the block's rows)
+  auto fetch = [&](int64_t tt, int slot) {
+    if (tt < t_end) cp_async16(rbase + (uint32_t)(slot * kThreads * 16), xc + (size_t)tt * a.channels);
+    cp_async_commit();
+  };
+#pragma unroll
+  for (int u = 0; u + 1 < kDepth; ++u) fetch(t_begin + u, u);
   float w[K][E], b[E];
   load_taps<E, K>(a, c0, w, b);
-  const IO* x = static_cast<const IO*>(a.x);
   int n = a.cu ? seq_of(a.cu, a.num_seqs, t_begin) : (int)(t_begin / a.uniform_len);
   int64_t s_begin, s_end;
   seq_bounds(a.cu, a.uniform_len, n, s_begin, s_end);
@@ -145,59 +172,50 @@ __global__ void __launch_bounds__(kThreads) conv_fwd_kernel(ConvArgs a) {
   for (int j = 0; j + 1 < K; ++j) {
     const int64_t p = t_begin - (K - 1) + j;
     if (p >= s_begin) {
-      unpack16<IO>(ld16(x + (size_t)p * a.channels + c0), win[j]);
+      unpack16<IO>(ld16(xc + (size_t)p * a.channels), win[j]);
     } else {
 #pragma unroll
       for (int e = 0; e < E; ++e) win[j][e] = window_at<IO>(a, n, c0 + e, (int)(K + (p - s_begin)));
     }
   }
-  // double-buffered: the next kBatch rows are requested before the current ones are used
-  uint4 cur[kBatch], nxt[kBatch];
+  const int rows = (int)(t_end - t_begin);
+#pragma unroll 4  // the window shifts become register renames
+  for (int i = 0; i < rows; ++i) {
+    const int64_t t = t_begin + i;
+    // refill the slot read in the previous iteration, then wait for row i
+    fetch(t + kDepth - 1, (i + kDepth - 1) % kDepth);
+    cp_async_wait<kDepth - 1>();
+    const uint4 raw = ring[(i % kDepth) * kThreads + threadIdx.x];
+    if (t >= s_end) {  // first token of the next non-empty sequence: restart the window
+      do {
+        ++n;
+        seq_bounds(a.cu, a.uniform_len, n, s_begin, s_end);
+      } while (t >= s_end);
 #pragma unroll
-  for (int u = 0; u < kBatch; ++u)
-    cur[u] = (t_begin + u < t_end) ? ld16(x + (size_t)(t_begin + u) * a.channels + c0) : make_uint4(0u, 0u, 0u, 0u);
-  for (int64_t t0 = t_begin; t0 < t_end; t0 += kBatch) {
+      for (int j = 0; j + 1 < K; ++j)
 #pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int64_t tn = t0 + kBatch + u;
-      nxt[u] = (tn < t_end) ? ld16(x + (size_t)tn * a.channels + c0) : make_uint4(0u, 0u, 0u, 0u);
+        for (int e = 0; e < E; ++e) win[j][e] = window_at<IO>(a, n, c0 + e, j + 1);
     }
+    float xt[E], acc[E];
+    unpack16<IO>(raw, xt);
 #pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int64_t t = t0 + u;
-      if (t >= t_end) break;
-      if (t >= s_end) {  // first token of the next non-empty sequence: restart the window
-        do {
-          ++n;
-          seq_bounds(a.cu, a.uniform_len, n, s_begin, s_end);
-        } while (t >= s_end);
+    for (int e = 0; e < E; ++e) {
+      float s_ = b[e];
 #pragma unroll
-        for (int j = 0; j + 1 < K; ++j)
-#pragma unroll
-          for (int e = 0; e < E; ++e) win[j][e] = window_at<IO>(a, n, c0 + e, j + 1);
-      }
-      float xt[E], acc[E];
-      unpack16<IO>(cur[u], xt);
-#pragma unroll
-      for (int e = 0; e < E; ++e) {
-        float s_ = b[e];
-#pragma unroll
-        for (int j = 0; j + 1 < K; ++j) s_ = fmaf(w[j][e], win[j][e], s_);
-        acc[e] = silu(fmaf(w[K - 1][e], xt[e], s_));
-      }
-      V16<IO>::store(out_ptr<IO>(a, t, c0), acc);
-#pragma unroll
-      for (int j = 0; j + 2 < K; ++j)
-#pragma unroll
-        for (int e = 0; e < E; ++e) win[j][e] = win[j + 1][e];
-      if (K > 1) {
-#pragma unroll
-        for (int e = 0; e < E; ++e) win[K > 1 ? K - 2 : 0][e] = xt[e];
-      }
+      for (int j = 0; j + 1 < K; ++j) s_ = fmaf(w[j][e], win[j][e], s_);
+      acc[e] = silu_io<IO>(fmaf(w[K - 1][e], xt[e], s_));
     }
+    V16<IO>::store(out_ptr<IO>(a, t, c0), acc);
 #pragma unroll
-    for (int u = 0; u < kBatch; ++u) cur[u] = nxt[u];
+    for (int j = 0; j + 2 < K; ++j)
+#pragma unroll
+      for (int e = 0; e < E; ++e) win[j][e] = win[j + 1][e];
+    if (K > 1) {
+#pragma unroll
+      for (int e = 0; e < E; ++e) win[K > 1 ? K - 2 : 0][e] = xt[e];
+    }
   }
+  cp_async_wait<0>();  // no copy outlives the block
 }
 
 // The conv_state after a prefill: the last K inputs of [window, sequence] of
@@ -262,7 +280,7 @@ __global__ void __launch_bounds__(kThreads) conv_update_kernel(ConvArgs a) {
     float acc = b[e];
 #pragma unroll
     for (int i = 0; i + 1 < K; ++i) acc = fmaf(w[i][e], win[e * K + i + 1], acc);
-    out[e] = silu(fmaf(w[K - 1][e], x[e], acc));
+    out[e] = silu_io<IO>(fmaf(w[K - 1][e], x[e], acc));
   }
   // the new window: shifted by one, the new input last
 #pragma unroll
@@ -282,8 +300,11 @@ static cudaError_t launch_fwd(const ConvArgs& a, cudaStream_t s) {
   const int vecs = a.channels / E;
   if (a.total_tokens > 0) {
     dim3 grid((unsigned)((a.total_tokens + kTokensPerBlock - 1) / kTokensPerBlock), (vecs + kThreads - 1) / kThreads);
-    conv_fwd_kernel<IO, K><<<grid, kThreads, 0, s>>>(a);
-    cudaError_t e = cudaGetLastError();
+    constexpr size_t smem = (size_t)kDepth * kThreads * 16;
+    cudaError_t e = cudaFuncSetAttribute(conv_fwd_kernel<IO, K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    conv_fwd_kernel<IO, K><<<grid, kThreads, smem, s>>>(a);
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   if (a.state_out) {

@@ -13,6 +13,7 @@
 // group.  A grid-stride loop over passes of U rows per lane group keeps the
 // grid at a multiple of the SM count.
 #include "gdn_common.cuh"
+#include "gdn_silu.cuh"
 #include "gdn_launch.h"
 
 namespace gdn {
@@ -97,7 +98,7 @@ __global__ void __launch_bounds__(kThreads) gated_rmsnorm_kernel(const IO* __res
         Vec<IO>::unpack(zw[u], zv);
         const float inv = rsqrtf(ss * (1.f / DIM) + eps);
 #pragma unroll
-        for (int e = 0; e < E; ++e) ov[e] = ov[e] * inv * wv[e] * silu(zv[e]);
+        for (int e = 0; e < E; ++e) ov[e] = ov[e] * inv * wv[e] * silu_io<IO>(zv[e]);
         Vec<IO>::store(y + (size_t)r * DIM + lane_in_row * E, ov);
       }
     }
