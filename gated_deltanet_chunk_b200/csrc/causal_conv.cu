@@ -294,6 +294,138 @@ __global__ void __launch_bounds__(kThreads) conv_update_kernel(ConvArgs a) {
   V16<IO>::store(out_ptr<IO>(a, n, c0), out);
 }
 
+// Decode update for K in {1, 2, 4}: a thread owns CH channels of kSeqPerThread
+// sequences, CH chosen so that its state span (CH channels x K taps) is one
+// 16-byte vector.  A warp's state loads and stores are then contiguous 512-byte
+// runs and its x / q, k, v accesses contiguous too, and the thread's taps (CH K
+// fp32: one or two 16-byte vectors) are loaded once for all its sequences.  The
+// kernel above spans 16 K bytes of state and 4 K floats of taps per thread, so a
+// warp-wide access touches 16 to 32 cache lines: its L1 data pipe, not DRAM,
+// set the pace (87 % busy, DRAM 12 %).  All sequences' loads are issued before
+// any is used.  The decode workload's update (256 sequences, 8192 channels,
+// 42 MB) measured 18.8 us with that kernel and 8.6 us with this one (2
+// sequences per thread; 4: 8.75 us, 8: 9.8 us), CUDA graphs on one box.
+constexpr int kSeqPerThread = 2;
+
+template <int B> __device__ __forceinline__ void ld_words(const void* p, uint32_t (&w)[B / 4]) {
+  if constexpr (B == 4) {
+    w[0] = *reinterpret_cast<const uint32_t*>(p);
+  } else if constexpr (B == 8) {
+    const uint2 v = *reinterpret_cast<const uint2*>(p);
+    w[0] = v.x; w[1] = v.y;
+  } else {
+    const uint4 v = *reinterpret_cast<const uint4*>(p);
+    w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+  }
+}
+template <int B> __device__ __forceinline__ void st_words(void* p, const uint32_t (&w)[B / 4]) {
+  if constexpr (B == 4) {
+    *reinterpret_cast<uint32_t*>(p) = w[0];
+  } else if constexpr (B == 8) {
+    *reinterpret_cast<uint2*>(p) = make_uint2(w[0], w[1]);
+  } else {
+    *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+// W 32-bit words <-> the 4 W / sizeof(IO) values of IO they hold (low half first)
+template <typename IO, int W> __device__ __forceinline__ void unpack_words(const uint32_t (&w)[W], float* x) {
+  if constexpr (sizeof(IO) == 4) {
+#pragma unroll
+    for (int i = 0; i < W; ++i) x[i] = __uint_as_float(w[i]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < W; ++i) {
+      x[2 * i] = __uint_as_float(w[i] << 16);
+      x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  }
+}
+template <typename IO, int W> __device__ __forceinline__ void pack_words(const float* x, uint32_t (&w)[W]) {
+  if constexpr (sizeof(IO) == 4) {
+#pragma unroll
+    for (int i = 0; i < W; ++i) w[i] = __float_as_uint(x[i]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < W; ++i) {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+      w[i] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+  }
+}
+
+template <typename IO, int K>
+__global__ void __launch_bounds__(kThreads) conv_update_packed_kernel(ConvArgs a) {
+  static_assert(K == 1 || K == 2 || K == 4, "the state span of CH channels is one 16-byte vector");
+  constexpr int ESZ = (int)sizeof(IO);
+  constexpr int CH = 16 / (K * ESZ);  // channels per thread
+  constexpr int XB = CH * ESZ;        // bytes of x and of the output per thread: 4, 8 or 16
+  const int c0 = (blockIdx.x * kThreads + threadIdx.x) * CH;
+  if (c0 >= a.channels) return;
+  float w[CH][K], b[CH];
+  {
+    const float4* wp = reinterpret_cast<const float4*>(a.weight + (size_t)c0 * K);  // CH K = 16 / ESZ floats
+#pragma unroll
+    for (int q = 0; q < CH * K / 4; ++q) {
+      const float4 v = __ldg(wp + q);
+      const float f[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int r = 0; r < 4; ++r) w[(4 * q + r) / K][(4 * q + r) % K] = f[r];
+    }
+#pragma unroll
+    for (int e = 0; e < CH; ++e) b[e] = a.bias ? __ldg(a.bias + c0 + e) : 0.f;
+  }
+  const int n0 = blockIdx.y * kSeqPerThread;
+  int64_t rows[kSeqPerThread];  // state row; -1 for a padding sequence, -2 past the batch
+  uint32_t xw[kSeqPerThread][XB / 4];
+  uint4 sw[kSeqPerThread];
+#pragma unroll
+  for (int s = 0; s < kSeqPerThread; ++s) {
+    const int n = n0 + s;
+    int64_t row = -2;
+    if (n < a.num_seqs) {
+      row = n;
+      if (a.slots) {
+        const int32_t id = a.slots[n];
+        row = (id >= 0 && id < a.num_slots) ? id : -1;
+      }
+    }
+    rows[s] = row;
+    if (row >= 0) {
+      ld_words<XB>(static_cast<const IO*>(a.x) + (size_t)n * a.channels + c0, xw[s]);
+      sw[s] = ld16(static_cast<const IO*>(a.state_out) + ((size_t)row * a.channels + c0) * K);
+    }
+  }
+#pragma unroll
+  for (int s = 0; s < kSeqPerThread; ++s) {
+    const int n = n0 + s;
+    if (rows[s] == -2) break;
+    float out[CH];
+    if (rows[s] >= 0) {
+      float x[CH], win[CH * K];  // window: channel e's entries at e K .. e K + K - 1, oldest first
+      unpack_words<IO, XB / 4>(xw[s], x);
+      unpack16<IO>(sw[s], win);
+#pragma unroll
+      for (int e = 0; e < CH; ++e) {
+        // taps 0..K-2 meet the window's entries 1..K-1, tap K-1 the new input
+        float acc = b[e];
+#pragma unroll
+        for (int i = 0; i + 1 < K; ++i) acc = fmaf(w[e][i], win[e * K + i + 1], acc);
+        out[e] = silu_io<IO>(fmaf(w[e][K - 1], x[e], acc));
+#pragma unroll
+        for (int i = 0; i + 1 < K; ++i) win[e * K + i] = win[e * K + i + 1];
+        win[e * K + K - 1] = x[e];
+      }
+      V16<IO>::store(static_cast<IO*>(a.state_out) + ((size_t)rows[s] * a.channels + c0) * K, win);
+    } else {
+#pragma unroll
+      for (int e = 0; e < CH; ++e) out[e] = 0.f;  // a padding sequence: zero output, no state
+    }
+    uint32_t ow[XB / 4];
+    pack_words<IO, XB / 4>(out, ow);
+    st_words<XB>(out_ptr<IO>(a, n, c0), ow);
+  }
+}
+
 template <typename IO, int K>
 static cudaError_t launch_fwd(const ConvArgs& a, cudaStream_t s) {
   constexpr int E = V16<IO>::N;
@@ -316,9 +448,15 @@ static cudaError_t launch_fwd(const ConvArgs& a, cudaStream_t s) {
 
 template <typename IO, int K>
 static cudaError_t launch_update(const ConvArgs& a, cudaStream_t s) {
-  constexpr int E = V16<IO>::N;
-  dim3 grid((a.channels / E + kThreads - 1) / kThreads, a.num_seqs);
-  conv_update_kernel<IO, K><<<grid, kThreads, 0, s>>>(a);
+  if constexpr (K == 3) {  // 3 taps x any channel count is no 16-byte span: a channel vector per thread
+    constexpr int E = V16<IO>::N;
+    dim3 grid((a.channels / E + kThreads - 1) / kThreads, a.num_seqs);
+    conv_update_kernel<IO, K><<<grid, kThreads, 0, s>>>(a);
+  } else {
+    constexpr int CH = 16 / (K * (int)sizeof(IO));
+    dim3 grid((a.channels / CH + kThreads - 1) / kThreads, (a.num_seqs + kSeqPerThread - 1) / kSeqPerThread);
+    conv_update_packed_kernel<IO, K><<<grid, kThreads, 0, s>>>(a);
+  }
   return cudaGetLastError();
 }
 

@@ -366,7 +366,7 @@ static int conv_common(const void* x, const float* weight, const float* bias, in
   if (num_seqs < 1 || num_seqs > 65535) return GDN_ERR_SHAPE;
   for (const void* ptr : {x, (const void*)q, (const void*)k, (const void*)v})
     if (ptr && !aligned16(ptr)) return GDN_ERR_ALIGN;
-  if (!aligned4(weight) || (bias && !aligned4(bias))) return GDN_ERR_ALIGN;
+  if (!aligned16(weight) || (bias && !aligned4(bias))) return GDN_ERR_ALIGN;  // taps move as 16-byte vectors
   a = gdn::ConvArgs{};
   a.x = x; a.weight = weight; a.bias = bias; a.num_seqs = num_seqs; a.ksize = kernel_size;
   a.nqk = p->num_qk_heads; a.nv = p->num_v_heads; a.dk = p->head_k_dim; a.dv = p->head_v_dim;

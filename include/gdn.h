@@ -307,7 +307,8 @@ int gdn_gated_rmsnorm(const void *o, const void *z, const float *weight, float e
  * newest at index K - 1.  All arithmetic is fp32; silu(x) = x / (1 + exp(-x)).
  *
  *   mixed_qkv   [T, C] (prefill, packed sequences) or [N, C] (decode), io_dtype
- *   weight      [C, K] fp32;  bias [C] fp32 or NULL (4-byte aligned)
+ *   weight      [C, K] fp32, 16-byte aligned (read as 16-byte vectors);
+ *               bias [C] fp32 or NULL, 4-byte aligned
  *   kernel_size K in [1, 4]
  *
  * gdn_qkv_conv_fwd (prefill over N sequences, cu_seqlens as in gdn_chunk_fwd):

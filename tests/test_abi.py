@@ -231,6 +231,7 @@ def test_conv_validation(L):
     assert fwd(pp=_p(nqk=3, nv=4)) == -2
     assert fwd(x=X + 8) == -3
     assert fwd(w=Wt + 2) == -3
+    assert fwd(w=Wt + 4) == -3                          # taps are read as 16-byte vectors
     assert fwd(q=X) == -4                               # q over the input
     assert fwd(k=Q + 4096) == -4                        # k over q
     assert fwd(si=A + 0x5000000, so=A + 0x5000000 + 64) == -4   # partial state overlap

@@ -73,11 +73,13 @@ def test_conv_fwd_in_place_state_and_equal_lengths():
     assert np.array_equal(U.to_np(st), ref_s)
 
 
+@pytest.mark.parametrize("K", [1, 2, 3, 4])
 @pytest.mark.parametrize("io", ["bf16", "f32"])
-def test_conv_update_equals_prefill_and_oracle(io):
-    """Per-token decode updates = one prefill over the same tokens; slot pool with padding rows."""
+def test_conv_update_equals_prefill_and_oracle(io, K):
+    """Per-token decode updates = one prefill over the same tokens; slot pool with padding rows.
+    N = 17 leaves a ragged last group of the sequences a thread takes (4)."""
     from gated_deltanet_chunk_b200 import qkv_conv_fwd, qkv_conv_update
-    nqk, nv, dk, dv, K, N, steps, P = 2, 4, 128, 128, 4, 16, 7, 40
+    nqk, nv, dk, dv, N, steps, P = 2, 4, 128, 128, 17, 7, 40
     c = W.make_conv_inputs(N * steps, nqk, nv, dk, dv, K, io, seed=73, num_states=P)
     x = c["x"].reshape(steps, N, c["C"])                    # token t of sequence n at x[t, n]
     ids = np.random.default_rng(73).permutation(P)[:N].astype(np.int32)
