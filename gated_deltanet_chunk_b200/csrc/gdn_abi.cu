@@ -65,7 +65,7 @@ float resolve_scale(const gdn_params_t* p) {
 
 }  // namespace
 
-GDN_API int gdn_version(void) { return (1 << 16) | 4; }
+GDN_API int gdn_version(void) { return (1 << 16) | 5; }
 
 GDN_API const char* gdn_status_string(int status) {
   switch (status) {
