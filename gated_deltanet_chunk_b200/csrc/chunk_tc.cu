@@ -16,7 +16,7 @@
 //     fp32 state slice S [128 x 64] lives in TMEM (lane d holds row d) and,
 //     rounded to bf16, in shared memory as the B operand of the next
 //     chunk.  The critical path per chunk is three tensor-core round trips
-//     ([K;Q] S with U, then V', then D4) and three short epilogues; W itself
+//     ([K;Q] S, then U and V', then D4) and three short epilogues; W itself
 //     is never formed.  P V' is issued by a second thread, so the thread that
 //     polls D4 goes straight from issuing it to waiting on it.  The output
 //     rows (P V' + Q S) are finished by warps 10-11 while warps 8-9 start the
@@ -37,7 +37,7 @@
 //        T = I + A T (one column per lane, one block per warp), then
 //        T_10 = T_11 (A_10 T_00) for both 32 x 32 blocks and
 //        T21 = T22 (A21 T11) for the whole, over all 256 intra threads
-//   serial:  U = T diag(beta) V,  [K S; Q S] = [K; Q] S                one round
+//   serial:  [K S; Q S] = [K; Q] S, then U = T diag(beta) V           one round
 //            K S rounded to bf16                                      CUDA cores
 //            V' = U + (-T diag(beta exp(gcum) rk)) (K S) = U - W S      one round
 //            D4 = K^T diag(rk exp(g_last - gcum)) V'                    one round
@@ -648,7 +648,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float* spp = sp + psl * SP_N;
       const uint32_t tm_qs = TM_QS + 64u * par;  // [K S; Q S] alternates between two column blocks
       if (vrow) {
-        // U = T diag(beta) V and [K S; Q S]
+        // [K S; Q S], committed alone so that the K S epilogue need not wait
+        // for U = T diag(beta) V, issued after it (the tensor pipe runs one
+        // thread's MMAs in order; the commit of the next round covers U)
         if (t == 0) {
           if (!ptx::mbar_wait_bounded(bars + BAR_RAWF + rsl, (uint32_t)((c / NR) & 1), kWaitNs) ||
               !ptx::mbar_wait_cluster_bounded(bars + BAR_PRODF + psl, (uint32_t)((c / NP) & 1), kWaitNs))
@@ -656,9 +658,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (*abort_flag == 0) {
             ptx::fence_proxy_async_smem();  // products stored by threads (possibly of the other CTA)
             ptx::tc_fence_after();
-            mma_k64(tmem + TM_U, pa + PS_TU, ra + RS_V, 8192, ID_KMN64, 0);
             mma_k128(tmem + tm_qs, ra + RS_KLO, ra + RS_KHI, sb + OFF_S, 8192, ID_KMN64, 0);
             ptx::mma_commit(bars + BAR_MMAW);
+            mma_k64(tmem + TM_U, pa + PS_TU, ra + RS_V, 8192, ID_KMN64, 0);
             if (!ptx::mbar_wait_bounded(bars + BAR_MMAW, par, kWaitNs)) *abort_flag = 1;
           }
         }
