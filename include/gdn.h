@@ -212,7 +212,9 @@ int gdn_recurrent_step_gated(const void *q, const void *k, const void *v,
  *   norm_eps         v-head) row o of Dv outputs is stored as
  *                        y = o / sqrt(mean(o^2) + norm_eps) * norm_weight * silu(z),
  *                        silu(x) = x / (1 + exp(-x)),
- *                    computed in fp32.  gdn_recurrent_step_ex normalises the fp32 o
+ *                    computed in fp32 (where gdn_chunk_fwd_ex's pass stores bf16,
+ *                    silu is evaluated as h + h tanh(h), h = x / 2, with the
+ *                    hardware tanh approximation: error at most |x| 2^-12).  gdn_recurrent_step_ex normalises the fp32 o
  *                    before its one rounding to io_dtype; gdn_chunk_fwd_ex stores o
  *                    and then rewrites each row in place (gdn_gated_rmsnorm), so
  *                    there o is rounded to io_dtype once before the norm.
@@ -283,6 +285,8 @@ int gdn_recurrent_step_ex(const void *q, const void *k, const void *v,
  *   weight    [dim] fp32, 16-byte aligned
  *   rows      >= 0 (< 2^31);  dim in {64, 128};  eps finite, >= 0.  With rows == 0
  *             the call does nothing and returns GDN_OK (the pointers may be NULL).
+ * Arithmetic is fp32; for bf16 io silu is evaluated as h + h tanh(h), h = x / 2,
+ * with the hardware tanh approximation (error at most |x| 2^-12).
  */
 int gdn_gated_rmsnorm(const void *o, const void *z, const float *weight, float eps,
                       void *y, int64_t rows, int32_t dim, int32_t io_dtype,
@@ -304,7 +308,10 @@ int gdn_gated_rmsnorm(const void *o, const void *z, const float *weight, float e
  * rest to v[t, c - 2 Nqk Dk]; q, k are [rows, Nqk, Dk] and v [rows, Nv, Dv] in
  * io_dtype, as gdn_chunk_fwd / gdn_recurrent_step read them.  A conv_state row
  * is [C, K] in io_dtype holding the last K inputs (pre-convolution), the
- * newest at index K - 1.  All arithmetic is fp32; silu(x) = x / (1 + exp(-x)).
+ * newest at index K - 1.  All arithmetic is fp32; silu(x) = x / (1 + exp(-x)),
+ * for bf16 io evaluated as h + h tanh(h), h = x / 2, with the hardware tanh
+ * approximation (error at most |x| 2^-12, under the rounding of a bf16 output
+ * for x > 0).
  *
  *   mixed_qkv   [T, C] (prefill, packed sequences) or [N, C] (decode), io_dtype
  *   weight      [C, K] fp32, 16-byte aligned (read as 16-byte vectors);
