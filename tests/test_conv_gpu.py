@@ -272,3 +272,34 @@ def test_fused_conv_norm_decode_full_shape_sampled():
         assert U.rel_inf(U.to_np(go[i]), o[i]) <= U.TOL["bf16"], pick_seqs[i]
     assert U.rel_inf(U.to_np(state[idx.cuda()]), sf) <= U.TOL["bf16"]
     assert np.array_equal(U.to_np(cst[idx.cuda()]), ref_cs)
+
+
+@pytest.mark.parametrize("io", ["bf16", "f32"])
+def test_silu_evaluation_error_bound(io):
+    """With the last tap 1, the others 0, no bias and an empty window, the conv is silu(x) itself.
+    Per element against x sigmoid(x) in fp64, over x in [-20, 20], in both the prefill and the
+    update kernels: bf16 outputs within their rounding (2^-8 relative) plus |x| 2^-12 (SiLU as
+    h + h tanh(h), h = x / 2, with tanh.approx's 2^-11 relative bound); fp32 outputs within
+    1e-5 relative (the exp / divide intrinsics)."""
+    from gated_deltanet_chunk_b200 import qkv_conv_fwd, qkv_conv_update
+    nqk, nv, d, K, T = 1, 1, 128, 4, 64
+    C = 2 * nqk * d + nv * d
+    dt = torch.bfloat16 if io == "bf16" else torch.float32
+    x = torch.linspace(-20.0, 20.0, T * C, dtype=torch.float64).reshape(T, C).to(dt)
+    w = torch.zeros(C, K, dtype=torch.float32)
+    w[:, K - 1] = 1.0
+    xd = x.double().numpy()
+    ref = xd / (1.0 + np.exp(-xd))
+    if io == "bf16":
+        bound = 2.0 ** -8 * np.abs(ref) + 1.01 * 2.0 ** -12 * np.abs(xd) + 1e-30
+    else:
+        bound = 1e-5 * np.abs(ref) + 1e-30
+    q, k, v, _ = qkv_conv_fwd(x.cuda(), w.cuda(), nqk, nv, d, d, num_seqs=1, output_state=False)
+    state = torch.zeros(T, C, K, dtype=dt, device="cuda")
+    q2, k2, v2 = qkv_conv_update(x.cuda(), w.cuda(), state, nqk, nv, d, d)
+    torch.cuda.synchronize()
+    for what, parts in (("prefill", (q, k, v)), ("update", (q2, k2, v2))):
+        y = torch.cat([p_.reshape(T, -1) for p_ in parts], 1).double().cpu().numpy()
+        err = np.abs(y - ref)
+        worst = int(np.argmax(err / bound))
+        assert np.all(err <= bound), (what, float(xd.flat[worst]), float(y.flat[worst]), float(ref.flat[worst]))
