@@ -26,30 +26,17 @@ namespace gdn {
 namespace conv {
 
 constexpr int kThreads = 256;
-constexpr int kTokensPerBlock = 128;  // prefill: consecutive tokens per thread (64: 0.517 ms, 32: 0.562 ms)
+constexpr int kTokensPerBlock = 128;  // prefill: consecutive tokens per thread (64 and 32 measured slower)
 
 template <typename IO> struct V16;
 template <> struct V16<float> {
   static constexpr int N = 4;
-  __device__ static void load(const void* p, float* x) {
-    const float4 v = *reinterpret_cast<const float4*>(p);
-    x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
-  }
   __device__ static void store(void* p, const float* x) {
     *reinterpret_cast<float4*>(p) = make_float4(x[0], x[1], x[2], x[3]);
   }
 };
 template <> struct V16<__nv_bfloat16> {
   static constexpr int N = 8;
-  __device__ static void load(const void* p, float* x) {
-    const uint4 v = *reinterpret_cast<const uint4*>(p);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      x[2 * i] = __uint_as_float(w[i] << 16);
-      x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-    }
-  }
   __device__ static void store(void* p, const float* x) {
     uint32_t w[4];
 #pragma unroll
