@@ -36,6 +36,30 @@ def test_every_declared_symbol_is_exported(L):
         assert hasattr(L, n), n
 
 
+def test_header_is_plain_c_and_links(L, tmp_path):
+    """include/gdn.h is a C header (no torch or C++ types): a C99 file that calls every declared
+    entry point compiles with -Wall -Werror and links against libgdn.so with no undefined symbol."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    names = declared_functions()
+    src = tmp_path / "use_all.c"
+    src.write_text('#include "gdn.h"\n'
+                   "typedef void (*fn)(void);\n"
+                   "fn table[] = {" + ", ".join("(fn)%s" % n for n in names) + "};\n")
+    obj, lib = tmp_path / "use_all.o", tmp_path / "libuse.so"
+    cc = ["gcc", "-std=c99", "-Wall", "-Werror", "-fPIC", "-I", os.path.join(ROOT, "include"), "-c", str(src),
+          "-o", str(obj)]
+    r = subprocess.run(cc, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    libdir = os.path.join(ROOT, "gated_deltanet_chunk_b200")
+    ld = ["gcc", "-shared", "-o", str(lib), str(obj), "-L", libdir, "-lgdn", "-Wl,--no-undefined",
+          "-Wl,-rpath," + libdir]
+    r = subprocess.run(ld, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+
+
 def test_version_and_status_strings(L):
     assert L.gdn_version() >> 16 == 1
     for code in range(-7, 1):
