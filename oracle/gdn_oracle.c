@@ -49,7 +49,7 @@
  *   cu_seqlens int32 [N+1]   sequence n owns tokens [cu[n], cu[n+1])  ([PTO])
  *   v-head h reads qk-head h / (Nv/Nqk)  ([WT] 一(一)4 repeat_interleave)
  *
- * Readings where the pages are silent or garbled (same list in the design doc):
+ * Readings where the pages are silent or garbled:
  *   - eps sits inside the square root ([PTO] L2 归一化);
  *   - the query scale 1/sqrt(Dk) is applied after the norm ([WT] 5(1)a);
  *   - the output of token t uses the state after token t's own write ([WT] (2));
