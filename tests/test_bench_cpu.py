@@ -82,3 +82,22 @@ def test_source_hash_covers_the_kernel_files():
         for f in files:
             assert os.path.exists(os.path.join(ROOT, "gated_deltanet_chunk_b200", "csrc", f)), f
         assert len(bench.source_hash(kernel)) == 64
+
+
+def test_reference_arm_under_torchrun_two_ranks():
+    """The launch the scaling run uses (torchrun, 2 ranks): rank 0 alone prints the line, every rank
+    exits 0, and no process group is needed for the CPU oracle."""
+    import socket
+    with socket.socket() as s_:
+        s_.bind(("127.0.0.1", 0))
+        port = s_.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"),
+           "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3", "--ref-sample-tokens", "4"]
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=900, cwd=ROOT,
+                       env={**os.environ, "CUDA_VISIBLE_DEVICES": ""})
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [x for x in r.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
