@@ -367,6 +367,14 @@ def run_ours(args, world, rank, local):
                                  call="gdn_chunk_fwd (cu_seqlens, initial and final state)",
                                  gpu_launches=max(3, args.steps // 4))
         del wv, ov, sv
+    # the two fp32 configurations (1 x 256 tokens, D 64, chunk 64; 4 x 4096
+    # tokens, Nqk 4, Nv 8, D 128, chunk 128, initial states), each against the
+    # HBM roofline and against the TF32 tensor peak measured here
+    if not args.no_fp32:
+        tf32 = measure_tf32_peak(dev)
+        res["tf32_peak_tflops"] = tf32
+        for name in ("tiny_f32_d64", "batch_f32_d128"):
+            res[name] = run_fp32_config(name, args, world, rank, dev, stream, peaks, peak_src, tf32)
     # the same workload with the gated RMSNorm epilogue fused into the output
     # stores (gdn_chunk_fwd_ex), and the epilogue on its own (gdn_gated_rmsnorm)
     if not args.no_norm:
@@ -478,6 +486,69 @@ def run_ours(args, world, rank, local):
                                          "sequences, all %d v-heads (%.1f s wall)"
                                          % (t_sample, n, nv, dt)}
     return res
+
+
+def measure_tf32_peak(dev, n=8192, reps=10):
+    """Dense fp32-in / fp32-out matmul throughput with TF32 tensor cores (torch, best of ``reps``, CUDA
+    events): the denominator of the fp32 configurations' tensor roofline (TFLOP/s)."""
+    import torch
+    prev = torch.backends.cuda.matmul.allow_tf32
+    torch.backends.cuda.matmul.allow_tf32 = True
+    try:
+        a = torch.randn(n, n, device=dev)
+        b = torch.randn(n, n, device=dev)
+        c = torch.empty(n, n, device=dev)
+        best = float("inf")
+        for _ in range(3):
+            torch.matmul(a, b, out=c)
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch.matmul(a, b, out=c)
+            e1.record()
+            torch.cuda.synchronize(dev)
+            best = min(best, e0.elapsed_time(e1))
+        del a, b, c
+        return 2.0 * n ** 3 / (best / 1e3) / 1e12
+    finally:
+        torch.backends.cuda.matmul.allow_tf32 = prev
+
+
+def run_fp32_config(name, args, world, rank, dev, stream, peaks, peak_src, tf32_tflops):
+    """One fp32 configuration: device time per gdn_chunk_fwd (CUDA events), tokens/s and both roofline terms."""
+    import torch
+
+    import gated_deltanet_chunk_b200 as gdn
+    import workloads as W
+    wl = W.WORKLOADS[name]
+    host = W.make_workload(name, seed=W.WORKLOAD_ORDER.index(name) + 10 * rank)
+    d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in host.items()}
+    n, T = wl.num_seqs, host["T"]
+    out = torch.empty(T, wl.nv, wl.d, dtype=torch.float32, device=dev)
+    sf = torch.empty(n, wl.nv, wl.d, wl.d, dtype=torch.float32, device=dev)
+
+    def step():
+        gdn.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["initial_state"], d["cu_seqlens"],
+                      chunk_size=wl.chunk, out=out, final_state=sf, kernel=args.kernel)
+
+    steps = max(10, args.steps)
+    ms = time_steps(step, args.warmup, steps, stream, world, dev)
+    byts = prefill_bytes(T, wl.nqk, wl.nv, wl.d, wl.d, n, 4, s0=wl.init_state, sf=True)
+    _, fl_tri = prefill_flops(T // n, n, wl.nv, wl.chunk, wl.d)
+    t_bytes = byts / (peaks["hbm_gbs"] * 1e9)
+    t_flops = fl_tri / (tf32_tflops * 1e12)
+    gbs = byts / (ms / 1e3) / 1e9
+    return {"value": T * world / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms, "workload": name,
+            "num_seqs": n, "seq_len": T // n, "nqk": wl.nqk, "nv": wl.nv, "d": wl.d, "chunk": wl.chunk,
+            "io": "f32", "initial_state": "random" if wl.init_state else "zeros",
+            "call": "gdn_chunk_fwd", "gpu_launches": steps,
+            "l2": "inputs below L2 size: repeated launches re-read them from L2 (an upper bound on speed)",
+            "roofline": {"bound": "hbm" if t_bytes >= t_flops else "tensor",
+                         "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": max(t_bytes, t_flops) / (ms / 1e3), "traffic": None, "peak_source": peak_src,
+                         "alg_bytes_per_launch": byts, "flops_tri_per_launch": fl_tri,
+                         "tf32_peak_tflops_measured": tf32_tflops,
+                         "roofline_time_ms": max(t_bytes, t_flops) * 1e3}}
 
 
 def run_decode(args, world, rank, dev, stream, peaks, peak_src):
@@ -663,7 +734,9 @@ def run_reference(args, world, rank):
             "data": "synthetic (seeded; workloads/)",
             "config": {"workload": PREFILL, "num_seqs": wl.num_seqs, "seq_len": wl.seq_len,
                        "nqk": wl.nqk, "nv": wl.nv, "dk": wl.d, "dv": wl.d, "chunk": wl.chunk,
-                       "io": "bf16", "parallelism": "host cores"},
+                       "io": "bf16", "state": "fp32", "initial_state": "zeros",
+                       "l2": "host run (no GPU cache involved)", "parallelism": "host cores",
+                       "sample_tokens_per_seq": args.ref_sample_tokens},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -687,6 +760,8 @@ def main():
     ap.add_argument("--no-gated", action="store_true", help="skip the fused-gate prefill and decode lines")
     ap.add_argument("--no-slots", action="store_true", help="skip the slot-indexed decode line")
     ap.add_argument("--no-varlen", action="store_true", help="skip the varlen prefill line")
+    ap.add_argument("--no-fp32", action="store_true",
+                    help="skip the lines of the two fp32 configurations (and the TF32 peak)")
     ap.add_argument("--no-conv", action="store_true",
                     help="skip the causal-conv lines (prefill conv, decode conv update)")
     ap.add_argument("--no-norm", action="store_true",

@@ -28,7 +28,7 @@ LIB_PATH = os.path.join(_HERE, "libgdn.so")
 GDN_OK = 0
 STATUS_NAMES = {0: "GDN_OK", -1: "GDN_ERR_NULL", -2: "GDN_ERR_SHAPE", -3: "GDN_ERR_ALIGN",
                 -4: "GDN_ERR_ALIAS", -5: "GDN_ERR_CUDA", -6: "GDN_ERR_DEVICE",
-                -7: "GDN_ERR_DEVICE_TIMEOUT"}
+                -7: "GDN_ERR_DEVICE_TIMEOUT", -8: "GDN_ERR_SEQLENS", -9: "GDN_ERR_GATE"}
 KERNELS = {"auto": 0, "simt": 1, "tc": 2}
 DTYPE_F32, DTYPE_BF16 = 0, 1
 

@@ -92,7 +92,7 @@ __device__ __forceinline__ IO* out_ptr(const ConvArgs& a, int64_t t, int c0) {
 // Channel c of the window before sequence n: conv_state[row, c, j], j in [0, K).
 template <typename IO>
 __device__ __forceinline__ float window_at(const ConvArgs& a, int64_t row, int c, int j) {
-  if (a.state_in == nullptr || row < 0) return 0.f;
+  if (a.state_in == nullptr || row < 0 || j < 0 || j >= a.ksize) return 0.f;
   return to_f32(static_cast<const IO*>(a.state_in)[((size_t)row * a.channels + c) * a.ksize + j]);
 }
 
@@ -152,7 +152,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSM) conv_fwd_kernel(ConvAr
   load_taps<E, K>(a, c0, w, b);
   int n = a.cu ? seq_of(a.cu, a.num_seqs, t_begin) : (int)(t_begin / a.uniform_len);
   int64_t s_begin, s_end;
-  seq_bounds(a.cu, a.uniform_len, n, s_begin, s_end);
+  seq_bounds(a, n, s_begin, s_end);
   // win[j] = input at position t - (K - 1) + j for the next token t
   float win[K > 1 ? K - 1 : 1][E];
 #pragma unroll
@@ -174,15 +174,17 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSM) conv_fwd_kernel(ConvAr
     cp_async_wait<kDepth - 1>();
     const uint4 raw = ring[(i % kDepth) * kThreads + threadIdx.x];
     if (t >= s_end) {  // first token of the next non-empty sequence: restart the window
-      do {
+      while (t >= s_end && n + 1 < a.num_seqs) {
         ++n;
-        seq_bounds(a.cu, a.uniform_len, n, s_begin, s_end);
-      } while (t >= s_end);
+        seq_bounds(a, n, s_begin, s_end);
+      }
 #pragma unroll
       for (int j = 0; j + 1 < K; ++j)
 #pragma unroll
         for (int e = 0; e < E; ++e) win[j][e] = window_at<IO>(a, n, c0 + e, j + 1);
     }
+    // a token of no sequence (only with inconsistent cu_seqlens, already reported) is not stored
+    const bool outside = t < s_begin || t >= s_end;
     float xt[E], acc[E];
     unpack16<IO>(raw, xt);
 #pragma unroll
@@ -192,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSM) conv_fwd_kernel(ConvAr
       for (int j = 0; j + 1 < K; ++j) s_ = fmaf(w[j][e], win[j][e], s_);
       acc[e] = silu_io<IO>(fmaf(w[K - 1][e], xt[e], s_));
     }
-    V16<IO>::store(out_ptr<IO>(a, t, c0), acc);
+    if (!outside) V16<IO>::store(out_ptr<IO>(a, t, c0), acc);
 #pragma unroll
     for (int j = 0; j + 2 < K; ++j)
 #pragma unroll
@@ -214,7 +216,7 @@ __global__ void __launch_bounds__(kThreads) conv_state_kernel(ConvArgs a) {
   if (idx >= (int64_t)a.num_seqs * a.channels) return;
   const int n = (int)(idx / a.channels), c = (int)(idx % a.channels);
   int64_t s_begin, s_end;
-  seq_bounds(a.cu, a.uniform_len, n, s_begin, s_end);
+  seq_bounds(a, n, s_begin, s_end);
   const int64_t len = s_end - s_begin;
   float v[K];
 #pragma unroll

@@ -121,7 +121,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_simt_kernel(ChunkArgs a
   const int nv = a.nv, nqk = a.nqk;
 
   int64_t seq_start, seq_end;
-  seq_bounds(a.cu, a.uniform_len, n, seq_start, seq_end);
+  seq_bounds(a, n, seq_start, seq_end);
 
   float* S = sm + L::kS;
   float* KhT = sm + L::kKhT;

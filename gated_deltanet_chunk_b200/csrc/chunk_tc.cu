@@ -61,8 +61,6 @@
 namespace gdn {
 namespace tc {
 
-__device__ unsigned int g_status;  // bit 0: a bounded wait expired
-
 constexpr int C = 64;
 constexpr int DK = 128;
 constexpr int DVS = 64;        // Dv columns per CTA
@@ -217,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* sp = reinterpret_cast<float*>(sm + OFF_SCP);
 
   int64_t seq_start, seq_end;
-  seq_bounds(a.cu, a.uniform_len, n, seq_start, seq_end);
+  seq_bounds(a, n, seq_start, seq_end);
   const int nchunks = (int)((seq_end - seq_start + C - 1) / C);
 
   const uint32_t crank = ptx::cluster_ctarank();  // == slice
@@ -279,6 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t t0g = seq_start + (int64_t)crank * C + t;
       if (t < 64 && t0g < seq_end) {
         load_gate_t<kRawGate>(a, (size_t)t0g * nv + h, h, g_next, b_next);
+        if (!(g_next <= 0.f)) report_status(a.status, kStatusGate);  // the decay factoring needs g <= 0
       }
     }
 
@@ -310,6 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         b_next = 0.f;
         if (tn < seq_end) {
           load_gate_t<kRawGate>(a, (size_t)tn * nv + h, h, g_next, b_next);
+          if (!(g_next <= 0.f)) report_status(a.status, kStatusGate);
         }
       }
       wait_bar(bars + BAR_RAWF + rsl, (uint32_t)((c / NR) & 1));
@@ -585,7 +585,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       named_bar_n(1, 256);
       if (t == 0) ptx::mbar_arrive(bars + BAR_PRODF + psl);  // the other CTA's copy completes by transactions
     }
-    if (!ok && t == 0) atomicOr(&g_status, 1u);
+    if (!ok && t == 0) report_status(a.status, kStatusTimeout);
   } else {
     // =====================================================================
     // serial warps (8-11)
@@ -816,7 +816,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int cc = 0; cc < 8; ++cc) dst[cc] = make_float4(x[4 * cc], x[4 * cc + 1], x[4 * cc + 2], x[4 * cc + 3]);
       }
     }
-    if (!ok && t == 0) atomicOr(&g_status, 1u);
+    if (!ok && t == 0) report_status(a.status, kStatusTimeout);
   }
 
   // Every thread that issued MMAs (intra 0, serial 0 and 32) commits once more:
@@ -827,7 +827,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   ptx::cluster_sync_all();  // the other CTA no longer touches this CTA's shared memory
   if (warp == 0) {
-    if (lane == 0 && !ptx::mbar_wait_bounded(bars + BAR_DRAIN, 0u, kWaitNs)) atomicOr(&g_status, 1u);
+    if (lane == 0 && !ptx::mbar_wait_bounded(bars + BAR_DRAIN, 0u, kWaitNs)) report_status(a.status, kStatusTimeout);
     __syncwarp();
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, TM_COLS);
@@ -863,8 +863,8 @@ static bool make_map(CUtensorMap* m, const void* ptr, int heads, int64_t T) {
 
 }  // namespace tc
 
-bool chunk_tc_supported(int dk, int dv, int chunk, int io_bf16, int64_t total_tokens) {
-  return io_bf16 && dk == 128 && dv == 128 && chunk == 64 && total_tokens > 0;
+bool chunk_tc_supported(int dk, int dv, int chunk, int io_bf16) {
+  return io_bf16 && dk == 128 && dv == 128 && chunk == 64;
 }
 
 cudaError_t launch_chunk_tc(const ChunkArgs& a, int64_t total_tokens, cudaStream_t stream) {
@@ -896,26 +896,19 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int64_t total_tokens, cudaStream
 // Self-test of the failure detection: one CTA waits, with the same bounded
 // mbarrier wait the chunk kernel uses, on a barrier nothing arrives on; after
 // limit_ns it gives up and records the timeout in the status word.
-__global__ void selftest_wait_kernel(uint64_t limit_ns) {
+__global__ void selftest_wait_kernel(uint64_t limit_ns, unsigned int* status) {
   __shared__ uint64_t bar;
   if (threadIdx.x == 0) {
     ptx::mbar_init(&bar, 1);
     ptx::fence_mbar_init();
   }
   __syncthreads();
-  if (threadIdx.x == 0 && !ptx::mbar_wait_bounded(&bar, 0u, limit_ns)) atomicOr(&tc::g_status, 1u);
+  if (threadIdx.x == 0 && !ptx::mbar_wait_bounded(&bar, 0u, limit_ns)) report_status(status, kStatusTimeout);
 }
 
-cudaError_t launch_selftest_wait(uint64_t limit_ns, cudaStream_t s) {
-  selftest_wait_kernel<<<1, 32, 0, s>>>(limit_ns);
+cudaError_t launch_selftest_wait(uint64_t limit_ns, unsigned int* status, cudaStream_t s) {
+  selftest_wait_kernel<<<1, 32, 0, s>>>(limit_ns, status);
   return cudaGetLastError();
-}
-
-unsigned int chunk_tc_take_status() {
-  unsigned int v = 0, zero = 0;
-  if (cudaMemcpyFromSymbol(&v, tc::g_status, sizeof(v)) != cudaSuccess) return ~0u;
-  if (v) cudaMemcpyToSymbol(tc::g_status, &zero, sizeof(zero));
-  return v;
 }
 
 }  // namespace gdn

@@ -30,6 +30,27 @@ bool overlap(Range a, Range b) {
   return a.lo < b.hi && b.lo < a.hi;
 }
 
+// The device status word every kernel reports into (gdn::kStatus* bits), and
+// the word gdn_device_status reads it into.  The kernels get the word's device
+// address, looked up once per device (cudaGetSymbolAddress, current device).
+__device__ unsigned int g_status_word;
+__device__ unsigned int g_status_taken;
+
+unsigned int* status_word() {
+  static unsigned int* addr[kMaxDevices] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<unsigned int*>(p);
+  }
+  return addr[dev];
+}
+
+// Reads and clears the status word in one atomic step, in stream order.
+__global__ void take_status_kernel() { g_status_taken = atomicExch(&g_status_word, 0u); }
+
 // The library ships sm_100a code only: require a compute capability 10.0 device.
 int check_device() {
   static int ok[kMaxDevices] = {0};  // 0 unknown, 1 ok, -1 bad
@@ -65,7 +86,7 @@ float resolve_scale(const gdn_params_t* p) {
 
 }  // namespace
 
-GDN_API int gdn_version(void) { return (1 << 16) | 5; }
+GDN_API int gdn_version(void) { return (1 << 16) | 6; }
 
 GDN_API const char* gdn_status_string(int status) {
   switch (status) {
@@ -77,6 +98,9 @@ GDN_API const char* gdn_status_string(int status) {
     case GDN_ERR_CUDA: return "GDN_ERR_CUDA: a CUDA call or kernel launch failed";
     case GDN_ERR_DEVICE: return "GDN_ERR_DEVICE: the current device is not compute capability 10.0";
     case GDN_ERR_DEVICE_TIMEOUT: return "GDN_ERR_DEVICE_TIMEOUT: a bounded in-kernel wait expired";
+    case GDN_ERR_SEQLENS:
+      return "GDN_ERR_SEQLENS: cu_seqlens was not non-decreasing from 0 to total_tokens (rows outside were skipped)";
+    case GDN_ERR_GATE: return "GDN_ERR_GATE: a gate g > 0 or NaN reached the tensor-core kernel, which needs g <= 0";
     default: return "GDN: unknown status";
   }
 }
@@ -157,6 +181,8 @@ static int chunk_fwd_impl(const void* q, const void* k, const void* v, const flo
 
   rc = check_device();
   if (rc) return rc;
+  unsigned int* status = status_word();
+  if (!status) return GDN_ERR_CUDA;
 
   gdn::ChunkArgs a{};
   a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.A_log = A_log; a.dt_bias = dt_bias;
@@ -164,6 +190,8 @@ static int chunk_fwd_impl(const void* q, const void* k, const void* v, const flo
   a.slots = slots; a.num_slots = num_slots;
   a.uniform_len = cu_seqlens ? 0 : (int32_t)(total_tokens / num_seqs);
   a.num_seqs = num_seqs;
+  a.total_tokens = total_tokens;
+  a.status = status;
   a.nqk = p->num_qk_heads; a.nv = p->num_v_heads; a.dv = p->head_v_dim;
   a.qk_l2norm = p->qk_l2norm ? 1 : 0;
   a.scale = resolve_scale(p);
@@ -171,7 +199,7 @@ static int chunk_fwd_impl(const void* q, const void* k, const void* v, const flo
   cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
 
   const int bf16 = p->io_dtype == GDN_DTYPE_BF16;
-  const bool tc_ok = gdn::chunk_tc_supported(p->head_k_dim, p->head_v_dim, chunk_size, bf16, total_tokens);
+  const bool tc_ok = gdn::chunk_tc_supported(p->head_k_dim, p->head_v_dim, chunk_size, bf16);
   if (p->kernel == GDN_KERNEL_TC && !tc_ok) return GDN_ERR_SHAPE;
   // Both chunk kernels split Dv across CTAs and store o; the norm epilogue then
   // rewrites the rows in place (one HBM-bound pass).  Fused into the
@@ -179,7 +207,9 @@ static int chunk_fwd_impl(const void* q, const void* k, const void* v, const flo
   // update rows 64..127 of the state, so their epilogue sits on the serial chain.
   a.nz = nullptr;
   cudaError_t e;
-  if (tc_ok && p->kernel != GDN_KERNEL_SIMT)
+  // an empty batch reads no token and only carries the states over: the CUDA-core
+  // launcher does that for every kernel setting
+  if (tc_ok && p->kernel != GDN_KERNEL_SIMT && total_tokens > 0)
     e = gdn::launch_chunk_tc(a, total_tokens, stream);
   else
     e = gdn::launch_chunk_simt(a, p->head_k_dim, chunk_size, bf16, stream);
@@ -407,6 +437,8 @@ GDN_API int gdn_qkv_conv_fwd(const void* mixed_qkv, const float* weight, const f
     return GDN_ERR_ALIAS;
   rc = check_device();
   if (rc) return rc;
+  a.status = status_word();
+  if (!a.status) return GDN_ERR_CUDA;
   a.state_in = conv_state_in; a.state_out = conv_state_out; a.cu = cu_seqlens;
   a.uniform_len = cu_seqlens ? 0 : (int32_t)(total_tokens / num_seqs);
   a.total_tokens = total_tokens;
@@ -444,6 +476,8 @@ GDN_API int gdn_qkv_conv_update(const void* mixed_qkv, const float* weight, cons
     return GDN_ERR_ALIAS;
   rc = check_device();
   if (rc) return rc;
+  a.status = status_word();
+  if (!a.status) return GDN_ERR_CUDA;
   a.state_in = conv_state; a.state_out = conv_state; a.slots = slot_ids; a.num_slots = num_slots;
   a.total_tokens = num_seqs;
   const cudaError_t e =
@@ -455,14 +489,28 @@ GDN_API int gdn_selftest_wait_timeout(int64_t limit_us, void* cuda_stream) {
   if (limit_us < 1 || limit_us > 2000000) return GDN_ERR_SHAPE;
   const int rc = check_device();
   if (rc) return rc;
-  const cudaError_t e = gdn::launch_selftest_wait((uint64_t)limit_us * 1000u, static_cast<cudaStream_t>(cuda_stream));
+  unsigned int* status = status_word();
+  if (!status) return GDN_ERR_CUDA;
+  const cudaError_t e =
+      gdn::launch_selftest_wait((uint64_t)limit_us * 1000u, status, static_cast<cudaStream_t>(cuda_stream));
   return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
 GDN_API int gdn_device_status(void* cuda_stream) {
-  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(cuda_stream));
-  if (e != cudaSuccess) return GDN_ERR_CUDA;
-  const unsigned int st = gdn::chunk_tc_take_status();
-  if (st == ~0u) return GDN_ERR_CUDA;
-  return st ? GDN_ERR_DEVICE_TIMEOUT : GDN_OK;
+  const int rc = check_device();
+  if (rc) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  // read-and-clear on the device, in stream order, so that no report made
+  // between a read and a separate clear is lost
+  take_status_kernel<<<1, 1, 0, s>>>();
+  if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+  unsigned int* taken = nullptr;
+  if (cudaGetSymbolAddress(reinterpret_cast<void**>(&taken), g_status_taken) != cudaSuccess) return GDN_ERR_CUDA;
+  unsigned int st = 0;
+  if (cudaMemcpyAsync(&st, taken, sizeof(st), cudaMemcpyDeviceToHost, s) != cudaSuccess) return GDN_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return GDN_ERR_CUDA;
+  if (st & gdn::kStatusTimeout) return GDN_ERR_DEVICE_TIMEOUT;
+  if (st & gdn::kStatusSeqlens) return GDN_ERR_SEQLENS;
+  if (st & gdn::kStatusGate) return GDN_ERR_GATE;
+  return GDN_OK;
 }

@@ -10,6 +10,15 @@ namespace gdn {
 
 constexpr float kNormEps = 1e-6f;  // L2 norm eps, inside the square root
 
+// Bits of the device status word that gdn_device_status reads and clears.
+constexpr unsigned int kStatusTimeout = 1u;  // a bounded in-kernel wait expired
+constexpr unsigned int kStatusSeqlens = 2u;  // cu_seqlens inconsistent with [0, total_tokens]
+constexpr unsigned int kStatusGate = 4u;     // a gate g > 0 (or NaN) reached a kernel that needs g <= 0
+
+__device__ __forceinline__ void report_status(unsigned int* status, unsigned int bit) {
+  if (status) atomicOr(status, bit);
+}
+
 // Arguments of the chunked forward (gdn_chunk_fwd); pointers are device memory.
 struct ChunkArgs {
   const void* q;             // [T, Nqk, Dk]
@@ -27,6 +36,8 @@ struct ChunkArgs {
   float* s_final;            // [N, Nv, Dk, Dv] or nullptr
   int32_t uniform_len;       // sequence length when cu == nullptr
   int32_t num_seqs;
+  int64_t total_tokens;      // T: rows of the token tensors
+  unsigned int* status;      // device status word (kStatus* bits)
   int32_t nqk, nv, dv;
   int32_t qk_l2norm;
   float scale;
@@ -77,6 +88,7 @@ struct ConvArgs {
   int64_t total_tokens;
   int32_t channels, ksize;   // channels = 2 nqk dk + nv dv
   int32_t nqk, nv, dk, dv;
+  unsigned int* status;      // device status word (kStatus* bits)
   void* q;                   // [T or N, nqk, dk] outputs
   void* k;
   void* v;                   // [T or N, nv, dv]
@@ -150,15 +162,23 @@ __device__ __forceinline__ int64_t state_row(const Args& a, int n) {
 // divisor stays below the 2^126 limit of __fdividef (silu(-80) is -1.4e-33).
 __device__ __forceinline__ float silu(float x) { return __fdividef(x, 1.f + __expf(fminf(-x, 80.f))); }
 
-// Sequence bounds [start, end) of sequence n.
-__device__ __forceinline__ void seq_bounds(const int32_t* cu, int32_t uniform_len, int n,
-                                           int64_t& start, int64_t& end) {
-  if (cu) {
-    start = cu[n];
-    end = cu[n + 1];
+// Sequence bounds [start, end) of sequence n, clamped to 0 <= start <= end <=
+// total_tokens.  cu_seqlens must be non-decreasing with cu[0] = 0 and
+// cu[num_seqs] = total_tokens ([PTO] README, 参数说明: act_seq_len holds the
+// cumulative lengths).  A violation that this sequence sees (its own bounds out
+// of order or out of range, or a wrong first / last entry) is reported through
+// the status word, and the clamped bounds keep every access inside the tensors.
+template <class Args>
+__device__ __forceinline__ void seq_bounds(const Args& a, int n, int64_t& start, int64_t& end) {
+  if (a.cu) {
+    const int64_t s = a.cu[n], e = a.cu[n + 1], T = a.total_tokens;
+    const bool bad = s < 0 || e < s || e > T || (n == 0 && s != 0) || (n == a.num_seqs - 1 && e != T);
+    start = s < 0 ? 0 : (s > T ? T : s);
+    end = e < start ? start : (e > T ? T : e);
+    if (bad) report_status(a.status, kStatusSeqlens);
   } else {
-    start = (int64_t)n * uniform_len;
-    end = start + uniform_len;
+    start = (int64_t)n * a.uniform_len;
+    end = start + a.uniform_len;
   }
 }
 

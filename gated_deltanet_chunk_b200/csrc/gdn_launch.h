@@ -11,12 +11,11 @@ namespace gdn {
 cudaError_t launch_chunk_simt(const ChunkArgs& a, int dk, int chunk, int io_bf16, cudaStream_t s);
 
 // Tensor-core chunked forward (tcgen05 + TMA): bf16 io, Dk = Dv = 128, chunk 64.
-bool chunk_tc_supported(int dk, int dv, int chunk, int io_bf16, int64_t total_tokens);
+bool chunk_tc_supported(int dk, int dv, int chunk, int io_bf16);
 cudaError_t launch_chunk_tc(const ChunkArgs& a, int64_t total_tokens, cudaStream_t s);
-// Reads and clears the tensor-core kernel's device status word (bit 0: a bounded wait expired).
-unsigned int chunk_tc_take_status();
-// One CTA whose bounded wait on a barrier nothing arrives on expires after limit_ns.
-cudaError_t launch_selftest_wait(uint64_t limit_ns, cudaStream_t s);
+// One CTA whose bounded wait on a barrier nothing arrives on expires after
+// limit_ns and records kStatusTimeout in *status.
+cudaError_t launch_selftest_wait(uint64_t limit_ns, unsigned int* status, cudaStream_t s);
 
 // One-token decode step; dk, dv in {64,128}.
 cudaError_t launch_recurrent_step(const StepArgs& a, int dk, int dv, int io_bf16, cudaStream_t s);

@@ -62,9 +62,10 @@ def test_header_is_plain_c_and_links(L, tmp_path):
 
 def test_version_and_status_strings(L):
     assert L.gdn_version() >> 16 == 1
-    for code in range(-7, 1):
+    for code in range(-9, 1):
         s = L.gdn_status_string(code).decode()
-        assert s.startswith("GDN")
+        assert s.startswith("GDN") and "unknown" not in s
+    assert "SEQLENS" in L.gdn_status_string(-8).decode() and "GATE" in L.gdn_status_string(-9).decode()
     assert "unknown" in L.gdn_status_string(5).decode()
 
 

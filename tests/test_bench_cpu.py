@@ -30,6 +30,10 @@ def test_reference_arm_json_line():
     assert d["value"] > 0 and d["unit"] == "tokens/s" and d["higher_is_better"] is True
     assert d["steps"] == 1 and d["warmup"] == 3 and d["n_gpus"] == 1
     assert d["config"]["workload"] == bench.PREFILL
+    # the same workload keys as the GPU arm's line, plus the declared sample
+    for key in ("num_seqs", "seq_len", "nqk", "nv", "dk", "dv", "chunk", "io", "state", "initial_state"):
+        assert key in d["config"], key
+    assert d["config"]["sample_tokens_per_seq"] == 8
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}

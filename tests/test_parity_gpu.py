@@ -234,15 +234,17 @@ def test_max_num_seqs_decode():
     U.check_prefill(out, state, ref_o, ref_s, cu, U.TOL["bf16"], "max-seqs-decode")
 
 
-@pytest.mark.parametrize("io,d", [("bf16", 128), ("f32", 64)])
-def test_empty_batch_copies_states(io, d):
-    """total_tokens = 0 (three empty sequences): final_state = initial_state, bit for bit."""
+@pytest.mark.parametrize("io,d,kernel", [("bf16", 128, "auto"), ("bf16", 128, "tc"), ("bf16", 128, "simt"),
+                                         ("f32", 64, "auto")])
+def test_empty_batch_copies_states(io, d, kernel):
+    """total_tokens = 0 (three empty sequences): final_state = initial_state, bit for bit, for every
+    kernel setting (the tensor-core setting included)."""
     from gated_deltanet_chunk_b200 import chunk_fwd
     dtype = torch.bfloat16 if io == "bf16" else torch.float32
     e = lambda *shape: torch.empty(*shape, dtype=dtype, device="cuda")
     s0 = torch.randn(3, 2, d, d, generator=torch.Generator().manual_seed(96)).cuda()
     g0 = torch.empty(0, 2, device="cuda")
     out, sf = chunk_fwd(e(0, 1, d), e(0, 1, d), e(0, 2, d), g0, g0.clone(), s0,
-                        torch.zeros(4, dtype=torch.int32, device="cuda"), chunk_size=64)
+                        torch.zeros(4, dtype=torch.int32, device="cuda"), chunk_size=64, kernel=kernel)
     torch.cuda.synchronize()
     assert out.numel() == 0 and torch.equal(sf, s0)
