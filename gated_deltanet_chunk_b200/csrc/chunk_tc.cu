@@ -5,8 +5,7 @@
 // columns.  The two CTAs of a (sequence, v-head) form a cluster.  In each CTA:
 //
 //   intra warps (0-7): the state-independent part of a chunk -- gate cumsum,
-//     L2 norms, G = [K;Q] K^T, the A and P matrices and T = (I - A)^-1 (fp32,
-//     CUDA cores).
+//     L2 norms, G = [K;Q] K^T, the A and P matrices and T = (I - A)^-1.
 //     Chunk c is built only by cluster rank c % 2, which writes the products
 //     (-T diag(bw), P, T diag(beta), per-row scalars) into its own product slot
 //     and, with st.async into distributed shared memory, into the same slot of
@@ -32,11 +31,10 @@
 //   G  = [K; Q] K^T                                     tcgen05 M=128 N=64 K=128
 //   A  = -strictLower(diag(beta rk) (K K^T) diag(rk) * Gamma)          CUDA cores
 //   P  = diag(rq) (Q K^T) diag(rk) * Gamma  (lower incl. diagonal)      CUDA cores
-//   T  = (I - A)^-1, fp32 in shared memory:                          CUDA cores
-//        the four 16 x 16 diagonal blocks by forward substitution on
-//        T = I + A T (one column per lane, one block per warp), then
-//        T_10 = T_11 (A_10 T_00) for both 32 x 32 blocks and
-//        T21 = T22 (A21 T11) for the whole, over all 256 intra threads
+//   T  = (I - A)^-1: the four 16 x 16 diagonal blocks by forward substitution
+//        on T = I + A T in fp32 (one column per lane, one block per warp), then
+//        T_10 = T_11 (A_10 T_00) for both 32 x 32 blocks and T21 = T22 (A21 T11)
+//        for the whole, as TF32 warp MMAs with fp32 accumulation
 //   serial:  [K S; Q S] = [K; Q] S, then U = T diag(beta) V           one round
 //            K S rounded to bf16                                      CUDA cores
 //            V' = U + (-T diag(beta exp(gcum) rk)) (K S) = U - W S      one round
@@ -277,7 +275,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t t0g = seq_start + (int64_t)crank * C + t;
       if (t < 64 && t0g < seq_end) {
         load_gate_t<kRawGate>(a, (size_t)t0g * nv + h, h, g_next, b_next);
-        if (!(g_next <= 0.f)) report_status(a.status, kStatusGate);  // the decay factoring needs g <= 0
       }
     }
 
@@ -297,6 +294,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // gates: beta and the warp-local cumsum of g; prefetch the next chunk's gates
       if (t < 64) {
         float gv = g_next;
+        // checked here, a chunk after the load was issued, so the check does not wait for it
+        if (!(gv <= 0.f)) report_status(a.status, kStatusGate);  // the decay factoring needs g <= 0
         si[SI_BETA + t] = b_next;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -309,7 +308,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         b_next = 0.f;
         if (tn < seq_end) {
           load_gate_t<kRawGate>(a, (size_t)tn * nv + h, h, g_next, b_next);
-          if (!(g_next <= 0.f)) report_status(a.status, kStatusGate);
         }
       }
       wait_bar(bars + BAR_RAWF + rsl, (uint32_t)((c / NR) & 1));
@@ -430,15 +428,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       // only drive the count below zero; the phase cannot complete before this
       // arrival, and the previous phase completed before the slot was released)
       if (t == 64) ptx::mbar_arrive_expect_tx_remote(rbar, kPushBytes);
-      // T = (I - A)^-1 in fp32 on the CUDA cores, by blocks (A is strictly lower
-      // triangular, T unit lower triangular).  M holds A^T on entry; each T block
-      // is written over an A^T block that is no longer needed, ending with T11,
-      // T22 row-major in M's diagonal 32 x 32 blocks and T21 in block (0, 1).
-      //   1. the four 16 x 16 diagonal blocks, T = I + A T from the top, one per
-      //      warp (0, 1, 4, 5; one column per lane); meanwhile warps 2, 3, 6, 7
-      //      store P, whose rows they hold
+      // T = (I - A)^-1 by blocks (A is strictly lower triangular, T unit lower
+      // triangular).  M holds A^T on entry; each T block is written over an A^T
+      // block that is no longer needed, ending with T11, T22 row-major in M's
+      // diagonal 32 x 32 blocks (their upper right 16 x 16 still holds A^T and is
+      // read as zero) and T21 in block (0, 1).
+      //   1. the four 16 x 16 diagonal blocks in fp32 on the CUDA cores, T = I + A T
+      //      from the top, one per warp (0, 1, 4, 5; one column per lane);
+      //      meanwhile warps 2, 3, 6, 7 store P, whose rows they hold
       //   2. both 32 x 32 diagonal blocks: T_10 = T_11 (A_10 T_00) on 16 x 16 blocks
-      //   3. T21 = T22 (A21 T11) on 32 x 32 blocks, all 8 warps, 2 x 2 tiles
+      //   3. T21 = T22 (A21 T11) on 32 x 32 blocks
+      // Steps 2 and 3 are TF32 warp MMAs with fp32 accumulation (T is rounded to
+      // bf16 as an MMA operand afterwards, far coarser than TF32's 2^-11).
       if (krow) {
         const int b = (warp & 1) | ((warp >> 2) << 1);  // warps 0, 1, 4, 5 -> blocks 0..3
         float* mb = ms + 16 * b * MS_LD + 16 * b;       // row k of this block of M = column k of A_bb
@@ -475,72 +476,94 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::st_half_packed_remote(rpa + PS_P, rbar, r, hf, pk0);
       }
       named_bar_n(1, 256);
-      {
-        // 2. pair p (blocks 2p, 2p + 1): thread -> row i, columns j0, j0 + 1 of a 16 x 16 block
-        const int pr = t >> 7, idx = t & 127, i = idx >> 3, j0 = 2 * (idx & 7);
-        float* base = ms + 32 * pr * MS_LD + 32 * pr;
-        // Y = A_10 T_00:  A_10[i][k] = base[k][16 + i] (A^T),  T_00[k][j] = base[k][j]
-        float y0 = 0.f, y1 = 0.f;
+      // 2. both 32 x 32 diagonal blocks: T_10 = T_11 (A_10 T_00) on 16 x 16 blocks,
+      //    warps 0-3 = (pair, 8-column tile), TF32 warp MMAs; Y = A_10 T_00 is
+      //    kept where A^T is zero (rows 16..31, columns 0..15 of the pair's block)
+      //    and then overwritten by T_10
+      const int g8 = lane >> 2, t4 = lane & 3;
+      if (warp < 4) {
+        const int pp = warp >> 1, nt = warp & 1;
+        float* base = ms + 32 * pp * MS_LD + 32 * pp;
+        float y[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const float a10 = base[k * MS_LD + 16 + i];
-          const float2 t00 = *reinterpret_cast<const float2*>(base + k * MS_LD + j0);
-          y0 = fmaf(a10, t00.x, y0);
-          y1 = fmaf(a10, t00.y, y1);
+        for (int k0 = 0; k0 < 16; k0 += 8) {
+          uint32_t af[4], bf[2];
+          af[0] = ptx::to_tf32(base[(k0 + t4) * MS_LD + 16 + g8]);      // A_10[g][k] = M[k][16 + g]
+          af[1] = ptx::to_tf32(base[(k0 + t4) * MS_LD + 24 + g8]);
+          af[2] = ptx::to_tf32(base[(k0 + t4 + 4) * MS_LD + 16 + g8]);
+          af[3] = ptx::to_tf32(base[(k0 + t4 + 4) * MS_LD + 24 + g8]);
+          bf[0] = ptx::to_tf32(base[(k0 + t4) * MS_LD + 8 * nt + g8]);  // T_00[k][n]
+          bf[1] = ptx::to_tf32(base[(k0 + t4 + 4) * MS_LD + 8 * nt + g8]);
+          ptx::mma_tf32_16x8x8(y, af, bf);
         }
-        *reinterpret_cast<float2*>(base + (16 + i) * MS_LD + j0) = make_float2(y0, y1);  // over A^T's zero block
-        named_bar_n(1, 256);
-        // T_10 = T_11 Y:  T_11[i][k] = base[16 + i][16 + k],  Y[k][j] = base[16 + k][j]
-        float z0 = 0.f, z1 = 0.f;
+        float* yo = base + 16 * MS_LD + 8 * nt + 2 * t4;
+        yo[g8 * MS_LD] = y[0];
+        yo[g8 * MS_LD + 1] = y[1];
+        yo[(g8 + 8) * MS_LD] = y[2];
+        yo[(g8 + 8) * MS_LD + 1] = y[3];
+        __syncwarp();
+        float z[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const float t11 = base[(16 + i) * MS_LD + 16 + k];
-          const float2 yk = *reinterpret_cast<const float2*>(base + (16 + k) * MS_LD + j0);
-          z0 = fmaf(t11, yk.x, z0);
-          z1 = fmaf(t11, yk.y, z1);
+        for (int k0 = 0; k0 < 16; k0 += 8) {
+          uint32_t af[4], bf[2];
+          af[0] = ptx::to_tf32(base[(16 + g8) * MS_LD + 16 + k0 + t4]);  // T_11[g][k]
+          af[1] = ptx::to_tf32(base[(24 + g8) * MS_LD + 16 + k0 + t4]);
+          af[2] = ptx::to_tf32(base[(16 + g8) * MS_LD + 20 + k0 + t4]);
+          af[3] = ptx::to_tf32(base[(24 + g8) * MS_LD + 20 + k0 + t4]);
+          bf[0] = ptx::to_tf32(base[(16 + k0 + t4) * MS_LD + 8 * nt + g8]);  // Y[k][n]
+          bf[1] = ptx::to_tf32(base[(20 + k0 + t4) * MS_LD + 8 * nt + g8]);
+          ptx::mma_tf32_16x8x8(z, af, bf);
         }
-        named_bar_n(1, 256);  // every read of Y is done
-        *reinterpret_cast<float2*>(base + (16 + i) * MS_LD + j0) = make_float2(z0, z1);
-        // the upper right 16 x 16 of the 32 x 32 block (A_10^T, consumed) becomes T's zeros
-        *reinterpret_cast<float2*>(base + i * MS_LD + 16 + j0) = make_float2(0.f, 0.f);
+        __syncwarp();  // every lane has read Y
+        yo[g8 * MS_LD] = z[0];
+        yo[g8 * MS_LD + 1] = z[1];
+        yo[(g8 + 8) * MS_LD] = z[2];
+        yo[(g8 + 8) * MS_LD + 1] = z[3];
       }
       named_bar_n(1, 256);
+      // 3. T21 = T22 (A21 T11) on 32 x 32 blocks: warp -> (16-row tile mt, 8-column
+      //    tile nt); T11 and T22 hold A^T values above their diagonal 16 x 16
+      //    blocks, so their upper triangles are masked to T's zeros as they are read
       {
-        // 3. 32 x 32 blocks: thread -> rows i2, i2 + 1 and columns j2, j2 + 1
-        const int i2 = 2 * (t >> 4), j2 = 2 * (t & 15);
-        // Y = A21 T11:  A21[i][k] = M[k][32 + i],  T11[k][j] = M[k][j]
-        float y[2][2] = {};
+        const int mt = warp >> 2, nt = warp & 3;
+        const int ra0 = 16 * mt + g8, cb = 8 * nt + g8;
+        float y[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          const float2 a = *reinterpret_cast<const float2*>(ms + k * MS_LD + 32 + i2);
-          const float2 b = *reinterpret_cast<const float2*>(ms + k * MS_LD + j2);
-          y[0][0] = fmaf(a.x, b.x, y[0][0]); y[0][1] = fmaf(a.x, b.y, y[0][1]);
-          y[1][0] = fmaf(a.y, b.x, y[1][0]); y[1][1] = fmaf(a.y, b.y, y[1][1]);
+        for (int k0 = 0; k0 < 32; k0 += 8) {
+          uint32_t af[4], bf[2];
+          af[0] = ptx::to_tf32(ms[(k0 + t4) * MS_LD + 32 + ra0]);  // A21[i][k] = M[k][32 + i]
+          af[1] = ptx::to_tf32(ms[(k0 + t4) * MS_LD + 40 + ra0]);
+          af[2] = ptx::to_tf32(ms[(k0 + t4 + 4) * MS_LD + 32 + ra0]);
+          af[3] = ptx::to_tf32(ms[(k0 + t4 + 4) * MS_LD + 40 + ra0]);
+          const int kb0 = k0 + t4, kb1 = k0 + t4 + 4;
+          bf[0] = ptx::to_tf32(cb <= kb0 ? ms[kb0 * MS_LD + cb] : 0.f);  // T11[k][n], lower triangle
+          bf[1] = ptx::to_tf32(cb <= kb1 ? ms[kb1 * MS_LD + cb] : 0.f);
+          ptx::mma_tf32_16x8x8(y, af, bf);
         }
-#pragma unroll
-        for (int r2 = 0; r2 < 2; ++r2)
-          *reinterpret_cast<float2*>(ms + (32 + i2 + r2) * MS_LD + j2) = make_float2(y[r2][0], y[r2][1]);
+        float* yo = ms + (32 + ra0) * MS_LD + 8 * nt + 2 * t4;  // Y over A^T's zero block
+        yo[0] = y[0];
+        yo[1] = y[1];
+        yo[8 * MS_LD] = y[2];
+        yo[8 * MS_LD + 1] = y[3];
         named_bar_n(1, 256);
-        // T21 = T22 Y:  T22[i][k] = M[32 + i][32 + k],  Y[k][j] = M[32 + k][j]; into block (0, 1)
-        float z[2][2] = {};
+        float z[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int k4 = 0; k4 < 32; k4 += 4) {
-          const float4 a0 = *reinterpret_cast<const float4*>(ms + (32 + i2) * MS_LD + 32 + k4);
-          const float4 a1 = *reinterpret_cast<const float4*>(ms + (32 + i2 + 1) * MS_LD + 32 + k4);
-          const float av[2][4] = {{a0.x, a0.y, a0.z, a0.w}, {a1.x, a1.y, a1.z, a1.w}};
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const float2 b = *reinterpret_cast<const float2*>(ms + (32 + k4 + kk) * MS_LD + j2);
-#pragma unroll
-            for (int r2 = 0; r2 < 2; ++r2) {
-              z[r2][0] = fmaf(av[r2][kk], b.x, z[r2][0]);
-              z[r2][1] = fmaf(av[r2][kk], b.y, z[r2][1]);
-            }
-          }
+        for (int k0 = 0; k0 < 32; k0 += 8) {
+          uint32_t af[4], bf[2];
+          const int ka = k0 + t4, kb = k0 + t4 + 4;
+          af[0] = ptx::to_tf32(ka <= ra0 ? ms[(32 + ra0) * MS_LD + 32 + ka] : 0.f);  // T22[i][k], lower
+          af[1] = ptx::to_tf32(ka <= ra0 + 8 ? ms[(40 + ra0) * MS_LD + 32 + ka] : 0.f);
+          af[2] = ptx::to_tf32(kb <= ra0 ? ms[(32 + ra0) * MS_LD + 32 + kb] : 0.f);
+          af[3] = ptx::to_tf32(kb <= ra0 + 8 ? ms[(40 + ra0) * MS_LD + 32 + kb] : 0.f);
+          bf[0] = ptx::to_tf32(ms[(32 + ka) * MS_LD + cb]);  // Y[k][n]
+          bf[1] = ptx::to_tf32(ms[(32 + kb) * MS_LD + cb]);
+          ptx::mma_tf32_16x8x8(z, af, bf);
         }
-#pragma unroll
-        for (int r2 = 0; r2 < 2; ++r2)
-          *reinterpret_cast<float2*>(ms + (i2 + r2) * MS_LD + 32 + j2) = make_float2(z[r2][0], z[r2][1]);
+        float* zo = ms + ra0 * MS_LD + 32 + 8 * nt + 2 * t4;  // T21 into block (0, 1)
+        zo[0] = z[0];
+        zo[1] = z[1];
+        zo[8 * MS_LD] = z[2];
+        zo[8 * MS_LD + 1] = z[3];
       }
       named_bar_n(1, 256);  // T21 is in M
       // products: stored locally first (and made visible to this CTA's tensor
@@ -562,6 +585,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int v = 0; v < 8; ++v) {
             const float4 y = *reinterpret_cast<const float4*>(tr + 4 * v);
             x[4 * v] = y.x; x[4 * v + 1] = y.y; x[4 * v + 2] = y.z; x[4 * v + 3] = y.w;
+          }
+          if ((r >> 5) == hf) {  // a diagonal 32 x 32 block: T is zero above the diagonal
+            const int rl = r & 31;
+#pragma unroll
+            for (int cc = 0; cc < 32; ++cc) x[cc] = cc <= rl ? x[cc] : 0.f;
           }
         }
         float y[32];
