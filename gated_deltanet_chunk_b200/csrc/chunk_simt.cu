@@ -10,7 +10,8 @@
 //   o  = diag(exp(gcum)) Q S + P V',  P = (Q K^T * Gamma), lower incl. diagonal
 //   S <- exp(g_last) S + (K * exp(g_last - gcum))^T V'
 //
-// where T = (I - A)^-1 is obtained by the walkthrough's row recursion (step d),
+// where T = (I - A)^-1 (the walkthrough's step d, which forms it by a row
+// recursion; here by 16 x 16 diagonal blocks and doubling merges),
 // A = -strictLower(diag(beta) (K K^T * Gamma)), Gamma = exp(gcum_r - gcum_i)
 // for i <= r (mask before exp), gcum = in-chunk inclusive cumsum of g (step c).
 //
@@ -101,6 +102,68 @@ __device__ __forceinline__ void pair_matrix(float* sm, int tid) {
         }
         A[r * L::AP + i] = val;
       }
+  }
+}
+
+// T - I for T = (I - A)^-1, A strictly lower triangular (held in A, pitch AP),
+// written over A.  The walkthrough's row recursion (section 一(一)5(1) d) has
+// C - 1 dependent steps; here the same T comes from its block form:
+//   1. each 16 x 16 diagonal block by forward substitution, one warp per block
+//      and one column per lane: (T - I)[i][j] = A[i][j] + sum_{j<m<i} A[i][m] (T - I)[m][j];
+//   2. doubling the solved blocks, for s = 16, 32, ... < C: a diagonal block
+//      [[T00, 0], [T10, T11]] of size 2s has T10 = T11 A10 T00, formed as
+//      Y = A10 + A10 (T00 - I), then T10 = Y + (T11 - I) Y.
+// Y needs s x s floats per pair (C s / 2 in all), held in the V tile, which
+// is free until X is formed.
+template <int C, int DK>
+__device__ __forceinline__ void invert_blocked(float* sm, int tid) {
+  using L = Smem<C, DK>;
+  constexpr int AP = L::AP;
+  float* A = sm + L::kA;
+  float* Y = sm + L::kV;
+  static_assert(C / 16 <= kThreads / 32, "one warp per diagonal block");
+  static_assert(C * C / 4 <= C * kDVS, "Y fits in the V tile");
+  const int lane = tid & 31, warp = tid >> 5;
+  if (warp < C / 16 && lane < 16) {
+    float* blk = A + (16 * warp) * AP + 16 * warp;
+    const int jc = lane;
+    float x[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      float acc = (jc < i) ? blk[i * AP + jc] : 0.f;
+#pragma unroll
+      for (int m = 0; m < i; ++m)
+        if (m > jc) acc = fmaf(blk[i * AP + m], x[m], acc);
+      x[i] = acc;
+    }
+    __syncwarp(0x0000ffffu);
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (jc < i) blk[i * AP + jc] = x[i];
+  }
+  __syncthreads();
+#pragma unroll 1
+  for (int s = 16; s < C; s *= 2) {
+    const int n = (C / (2 * s)) * s * s;  // outputs of the level: pairs x s x s
+    for (int e = tid; e < n; e += kThreads) {
+      const int p = e / (s * s), i = (e / s) % s, jc = e % s;
+      const int base = 2 * s * p;
+      const float* arow = A + (base + s + i) * AP + base;  // row i of A10
+      float y = arow[jc];
+      for (int m = jc + 1; m < s; ++m) y = fmaf(arow[m], A[(base + m) * AP + base + jc], y);
+      Y[e] = y;
+    }
+    __syncthreads();
+    for (int e = tid; e < n; e += kThreads) {
+      const int p = e / (s * s), i = (e / s) % s, jc = e % s;
+      const int base = 2 * s * p;
+      const float* trow = A + (base + s + i) * AP + base + s;  // row i of T11 - I
+      const float* yp = Y + p * s * s;
+      float t = yp[i * s + jc];
+      for (int m = 0; m < i; ++m) t = fmaf(trow[m], yp[m * s + jc], t);
+      A[(base + s + i) * AP + base + jc] = t;
+    }
+    __syncthreads();
   }
 }
 
@@ -207,21 +270,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_simt_kernel(ChunkArgs a
     // ---- A = -strictLower(diag(beta) (K K^T * Gamma)) ----
     pair_matrix<C, DK, false>(sm, tid);
     __syncthreads();
-    // ---- T - I by the row recursion  Tt_i = A_i + A_i Tt_{<i} ----
-    {
-      constexpr int TPJ = kThreads / C;  // threads per column
-      const int jc = tid / TPJ, part = tid % TPJ;
-      for (int i = 1; i < C; ++i) {
-        float val = 0.f;
-        if (jc < i)
-          for (int m = jc + 1 + part; m < i; m += TPJ) val = fmaf(A[i * L::AP + m], A[m * L::AP + jc], val);
-#pragma unroll
-        for (int o = 1; o < TPJ; o <<= 1) val += __shfl_xor_sync(0xffffffffu, val, o);
-        __syncthreads();
-        if (jc < i && part == 0) A[i * L::AP + jc] += val;
-        __syncthreads();
-      }
-    }
+    // ---- T - I by blocks, in place over A (strictly lower) ----
+    invert_blocked<C, DK>(sm, tid);
     // ---- X = diag(beta) (V - diag(exp(gcum)) K S) ----
     constexpr int NTV = (C / 4) * (kDVS / 4);
     for (int tile = tid; tile < NTV; tile += kThreads) {
