@@ -59,6 +59,32 @@ __device__ __forceinline__ float4 ld4_t(const float* base, int d, int r0) {
   return *reinterpret_cast<const float4*>(base + swz<C>(d, r0));
 }
 
+// PER consecutive elements of one row (from a 4 * PER-byte or 2 * PER-byte
+// aligned address) as fp32; zeros for a row past the sequence end.
+template <typename IO, int PER>
+__device__ __forceinline__ void load_row_part(const IO* p, bool valid, float* x) {
+  if (!valid) {
+#pragma unroll
+    for (int e = 0; e < PER; ++e) x[e] = 0.f;
+    return;
+  }
+  if constexpr (sizeof(IO) == 4 && PER == 4) {
+    const float4 y = *reinterpret_cast<const float4*>(p);
+    x[0] = y.x; x[1] = y.y; x[2] = y.z; x[3] = y.w;
+  } else if constexpr (sizeof(IO) == 4 && PER == 2) {
+    const float2 y = *reinterpret_cast<const float2*>(p);
+    x[0] = y.x; x[1] = y.y;
+  } else if constexpr (sizeof(IO) == 2 && PER == 4) {
+    const uint2 y = *reinterpret_cast<const uint2*>(p);
+    const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&y.x));
+    const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&y.y));
+    x[0] = lo.x; x[1] = lo.y; x[2] = hi.x; x[3] = hi.y;
+  } else {
+#pragma unroll
+    for (int e = 0; e < PER; ++e) x[e] = to_f32(p[e]);
+  }
+}
+
 // A (IS_P = false):  A[r][i] = -beta_r (k_r . k_i) Gamma[r][i] for i < r, else 0.
 // P (IS_P = true):   P[r][i] = (q_r . k_i) Gamma[r][i] for i <= r, else 0.
 template <int C, int DK, bool IS_P>
@@ -69,15 +95,21 @@ __device__ __forceinline__ void pair_matrix(float* sm, int tid) {
   const float* gc = sm + L::kGc;
   const float* bt = sm + L::kBeta;
   float* A = sm + L::kA;
-  constexpr int NTC = C / 4;
-  for (int tile = tid; tile < NTC * NTC; tile += kThreads) {
-    const int r0 = (tile / NTC) * 4, i0 = (tile % NTC) * 4;
+  // Only the 4 x 4 tiles on or below the diagonal are formed (numbered row by
+  // row: tile tl is (rt, it) with tl = rt (rt + 1) / 2 + it, it <= rt); no later
+  // step reads A or P above the diagonal tiles.
+  constexpr int NTC = C / 4, NL = NTC * (NTC + 1) / 2;
+  for (int tl = tid; tl < NL; tl += kThreads) {
+    int rt = (int)((sqrtf(8.f * (float)tl + 1.f) - 1.f) * 0.5f);
+    while ((rt + 1) * (rt + 2) / 2 <= tl) ++rt;
+    while (rt * (rt + 1) / 2 > tl) --rt;
+    const int r0 = rt * 4, i0 = (tl - rt * (rt + 1) / 2) * 4;
     float acc[4][4];
 #pragma unroll
     for (int a = 0; a < 4; ++a)
 #pragma unroll
       for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
-    if (i0 <= r0 + 3) {
+    {
 #pragma unroll 4
       for (int d = 0; d < DK; ++d) {
         const float4 x = ld4_t<C>(X, d, r0);
@@ -144,24 +176,64 @@ __device__ __forceinline__ void invert_blocked(float* sm, int tid) {
   __syncthreads();
 #pragma unroll 1
   for (int s = 16; s < C; s *= 2) {
-    const int n = (C / (2 * s)) * s * s;  // outputs of the level: pairs x s x s
-    for (int e = tid; e < n; e += kThreads) {
-      const int p = e / (s * s), i = (e / s) % s, jc = e % s;
+    // one 4 x 4 tile of the level's outputs per thread and pass
+    const int ts = s / 4, ntile = (C / (2 * s)) * ts * ts;
+    for (int e = tid; e < ntile; e += kThreads) {
+      const int p = e / (ts * ts), i0 = 4 * ((e / ts) % ts), j0 = 4 * (e % ts);
       const int base = 2 * s * p;
-      const float* arow = A + (base + s + i) * AP + base;  // row i of A10
-      float y = arow[jc];
-      for (int m = jc + 1; m < s; ++m) y = fmaf(arow[m], A[(base + m) * AP + base + jc], y);
-      Y[e] = y;
+      const float* a10 = A + (base + s) * AP + base;  // A10[i][m] = a10[i * AP + m]
+      const float* t00 = A + base * AP + base;        // (T00 - I)[m][j], zero for m <= j
+      float acc[4][4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[r][c] = a10[(i0 + r) * AP + j0 + c];
+#pragma unroll 4
+      for (int m = j0 + 1; m < s; ++m) {
+        float x[4], y[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) x[r] = a10[(i0 + r) * AP + m];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) y[c] = t00[m * AP + j0 + c];
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(x[r], y[c], acc[r][c]);
+      }
+      float* yp = Y + p * s * s;
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+        *reinterpret_cast<float4*>(yp + (i0 + r) * s + j0) = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
     }
     __syncthreads();
-    for (int e = tid; e < n; e += kThreads) {
-      const int p = e / (s * s), i = (e / s) % s, jc = e % s;
+    for (int e = tid; e < ntile; e += kThreads) {
+      const int p = e / (ts * ts), i0 = 4 * ((e / ts) % ts), j0 = 4 * (e % ts);
       const int base = 2 * s * p;
-      const float* trow = A + (base + s + i) * AP + base + s;  // row i of T11 - I
+      const float* t11 = A + (base + s) * AP + base + s;  // (T11 - I)[i][m], zero for m >= i
       const float* yp = Y + p * s * s;
-      float t = yp[i * s + jc];
-      for (int m = 0; m < i; ++m) t = fmaf(trow[m], yp[m * s + jc], t);
-      A[(base + s + i) * AP + base + jc] = t;
+      float acc[4][4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const float4 y = *reinterpret_cast<const float4*>(yp + (i0 + r) * s + j0);
+        acc[r][0] = y.x; acc[r][1] = y.y; acc[r][2] = y.z; acc[r][3] = y.w;
+      }
+#pragma unroll 4
+      for (int m = 0; m < i0 + 3; ++m) {
+        float x[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) x[r] = t11[(i0 + r) * AP + m];
+        const float4 y = *reinterpret_cast<const float4*>(yp + m * s + j0);
+        const float yv[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(x[r], yv[c], acc[r][c]);
+      }
+      float* t10 = A + (base + s) * AP + base;
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) t10[(i0 + r) * AP + j0 + c] = acc[r][c];
     }
     __syncthreads();
   }
@@ -206,29 +278,47 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_simt_kernel(ChunkArgs a
   for (int64_t c0 = seq_start; c0 < seq_end; c0 += C) {
     __syncthreads();  // previous chunk fully consumed
     // ---- load q, k rows; L2 norm (eps inside the root) and query scale ----
-    constexpr int PER = DK / 32;
-    for (int r = warp; r < C; r += kThreads / 32) {
-      const int64_t t = c0 + r;
-      const bool valid = t < seq_end;
-      float qv[PER], kv[PER];
-      float sq = 0.f, sk = 0.f;
+    // RB rows per warp at a time, so that their loads are in flight together
+    constexpr int PER = DK / 32, RB = 4;
+    static_assert(C % ((kThreads / 32) * RB) == 0, "rows per pass");
+    for (int r0 = warp * RB; r0 < C; r0 += (kThreads / 32) * RB) {
+      float qv[RB][PER], kv[RB][PER], sq[RB], sk[RB];
 #pragma unroll
-      for (int e = 0; e < PER; ++e) {
-        const size_t off = ((size_t)t * nqk + j) * DK + lane * PER + e;
-        qv[e] = valid ? to_f32(q[off]) : 0.f;
-        kv[e] = valid ? to_f32(k[off]) : 0.f;
-        sq += qv[e] * qv[e];
-        sk += kv[e] * kv[e];
+      for (int rb = 0; rb < RB; ++rb) {
+        const int64_t t = c0 + r0 + rb;
+        const bool valid = t < seq_end;
+        const size_t off = ((size_t)(valid ? t : 0) * nqk + j) * DK + lane * PER;
+        load_row_part<IO, PER>(q + off, valid, qv[rb]);
+        load_row_part<IO, PER>(k + off, valid, kv[rb]);
       }
-      sq = warp_sum(sq);
-      sk = warp_sum(sk);
-      const float fq = (a.qk_l2norm ? 1.f / sqrtf(sq + kNormEps) : 1.f) * a.scale;
-      const float fk = a.qk_l2norm ? 1.f / sqrtf(sk + kNormEps) : 1.f;
 #pragma unroll
-      for (int e = 0; e < PER; ++e) {
-        const int d = lane * PER + e;
-        QhT[swz<C>(d, r)] = qv[e] * fq;
-        KhT[swz<C>(d, r)] = kv[e] * fk;
+      for (int rb = 0; rb < RB; ++rb) {
+        sq[rb] = 0.f;
+        sk[rb] = 0.f;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) {
+          sq[rb] = fmaf(qv[rb][e], qv[rb][e], sq[rb]);
+          sk[rb] = fmaf(kv[rb][e], kv[rb][e], sk[rb]);
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int rb = 0; rb < RB; ++rb) {
+          sq[rb] += __shfl_xor_sync(0xffffffffu, sq[rb], o);
+          sk[rb] += __shfl_xor_sync(0xffffffffu, sk[rb], o);
+        }
+#pragma unroll
+      for (int rb = 0; rb < RB; ++rb) {
+        const int r = r0 + rb;
+        const float fq = (a.qk_l2norm ? 1.f / sqrtf(sq[rb] + kNormEps) : 1.f) * a.scale;
+        const float fk = a.qk_l2norm ? 1.f / sqrtf(sk[rb] + kNormEps) : 1.f;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) {
+          const int d = lane * PER + e;
+          QhT[swz<C>(d, r)] = qv[rb][e] * fq;
+          KhT[swz<C>(d, r)] = kv[rb][e] * fk;
+        }
       }
     }
     if (tid < C) {
