@@ -23,6 +23,7 @@
 // state unchanged.
 #include "gdn_common.cuh"
 #include "gdn_launch.h"
+#include "sm100_ptx.cuh"
 
 namespace gdn {
 namespace simt {
@@ -85,6 +86,41 @@ __device__ __forceinline__ void load_row_part(const IO* p, bool valid, float* x)
   }
 }
 
+// fp32 x = hi + lo with hi, lo both TF32 (the low 13 bits of each are zero):
+// products of such splits, hi hi + hi lo + lo hi, are within about 2^-22 of
+// the exact product, so three TF32 MMAs stand in for fp32 ones.  That is four
+// times fp32's rounding: the key-key and query-key dot products (A and P
+// below), whose cancellation sets the relative accuracy of short or nearly
+// orthogonal sequences' outputs, stay on fp32 FMAs.
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+  hi = ptx::to_tf32(x);
+  lo = ptx::to_tf32(x - __uint_as_float(hi));
+}
+
+// acc[NT] (16 x 8 fp32 tiles, columns 8 j .. 8 j + 7 of a 16 x 8 NT block) +=
+// A[16 x K] B[K x 8 NT] over k in [k0, k1) (multiples of 8), one warp, with
+// a(m, k) and b(k, n) reading the operands' elements (m < 16, n < 8 NT).
+template <int NT, typename FA, typename FB>
+__device__ __forceinline__ void warp_mma_3xtf32(float (&acc)[NT][4], int k0, int k1, FA a, FB b, int g, int t) {
+#pragma unroll 2
+  for (int kk = k0; kk < k1; kk += 8) {
+    uint32_t ah[4], al[4];
+    split_tf32(a(g, kk + t), ah[0], al[0]);
+    split_tf32(a(g + 8, kk + t), ah[1], al[1]);
+    split_tf32(a(g, kk + t + 4), ah[2], al[2]);
+    split_tf32(a(g + 8, kk + t + 4), ah[3], al[3]);
+#pragma unroll
+    for (int jj = 0; jj < NT; ++jj) {
+      uint32_t bh[2], bl[2];
+      split_tf32(b(kk + t, 8 * jj + g), bh[0], bl[0]);
+      split_tf32(b(kk + t + 4, 8 * jj + g), bh[1], bl[1]);
+      ptx::mma_tf32_16x8x8(acc[jj], al, bh);
+      ptx::mma_tf32_16x8x8(acc[jj], ah, bl);
+      ptx::mma_tf32_16x8x8(acc[jj], ah, bh);
+    }
+  }
+}
+
 // A (IS_P = false):  A[r][i] = -beta_r (k_r . k_i) Gamma[r][i] for i < r, else 0.
 // P (IS_P = true):   P[r][i] = (q_r . k_i) Gamma[r][i] for i <= r, else 0.
 template <int C, int DK, bool IS_P>
@@ -96,8 +132,14 @@ __device__ __forceinline__ void pair_matrix(float* sm, int tid) {
   const float* bt = sm + L::kBeta;
   float* A = sm + L::kA;
   // Only the 4 x 4 tiles on or below the diagonal are formed (numbered row by
-  // row: tile tl is (rt, it) with tl = rt (rt + 1) / 2 + it, it <= rt); no later
-  // step reads A or P above the diagonal tiles.
+  // row: tile tl is (rt, it) with tl = rt (rt + 1) / 2 + it, it <= rt).  The
+  // warp MMAs that read A (as T - I) and P take whole 16 x 16 diagonal blocks,
+  // so the entries above the diagonal tiles inside those blocks are zeroed;
+  // nothing reads further up.
+  for (int e = tid; e < (C / 16) * 256; e += kThreads) {
+    const int b = e >> 8, r = (e >> 4) & 15, i = e & 15;
+    if ((i >> 2) > (r >> 2)) A[(16 * b + r) * L::AP + 16 * b + i] = 0.f;
+  }
   constexpr int NTC = C / 4, NL = NTC * (NTC + 1) / 2;
   for (int tl = tid; tl < NL; tl += kThreads) {
     int rt = (int)((sqrtf(8.f * (float)tl + 1.f) - 1.f) * 0.5f);
@@ -362,138 +404,85 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_simt_kernel(ChunkArgs a
     __syncthreads();
     // ---- T - I by blocks, in place over A (strictly lower) ----
     invert_blocked<C, DK>(sm, tid);
+    // The products below are warp MMAs (TF32 split three ways) on 16 x 8 tiles:
+    // the C x 32 outputs (X, V', o) as C / 16 row blocks of four column tiles,
+    // and the DK x 32 state slice as DK / 16 row blocks, each warp taking
+    // consecutive tiles of one row block.
+    constexpr int NTV = C / 32;    // column tiles per warp for C-row outputs
+    constexpr int NTS = DK / 32;   // column tiles per warp for the state
+    const int g8 = lane >> 2, t4 = lane & 3;
+    const int vr0 = 16 * ((warp * NTV) / 4), vc0 = 8 * ((warp * NTV) % 4);  // this warp's C-row tiles
     // ---- X = diag(beta) (V - diag(exp(gcum)) K S) ----
-    constexpr int NTV = (C / 4) * (kDVS / 4);
-    for (int tile = tid; tile < NTV; tile += kThreads) {
-      const int r0 = (tile / (kDVS / 4)) * 4, cc0 = (tile % (kDVS / 4)) * 4;
-      float acc[4][4] = {};
-#pragma unroll 4
-      for (int d = 0; d < DK; ++d) {
-        const float4 x = ld4_t<C>(KhT, d, r0);
-        const float4 y = *reinterpret_cast<const float4*>(S + d * kDVS + cc0);
-        const float xs[4] = {x.x, x.y, x.z, x.w};
-        const float ys[4] = {y.x, y.y, y.z, y.w};
+    {
+      float acc[NTV][4] = {};
+      warp_mma_3xtf32<NTV>(acc, 0, DK,
+                           [&](int m, int kk) { return KhT[swz<C>(kk, vr0 + m)]; },
+                           [&](int kk, int n) { return S[kk * kDVS + vc0 + n]; }, g8, t4);
 #pragma unroll
-        for (int aa = 0; aa < 4; ++aa)
+      for (int jj = 0; jj < NTV; ++jj)
 #pragma unroll
-          for (int b = 0; b < 4; ++b) acc[aa][b] = fmaf(xs[aa], ys[b], acc[aa][b]);
-      }
-#pragma unroll
-      for (int aa = 0; aa < 4; ++aa) {
-        const int r = r0 + aa;
-        const int64_t t = c0 + r;
-        const bool valid = t < seq_end;
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          const float vv = valid ? to_f32(v[((size_t)t * nv + h) * dv + cslice + cc0 + b]) : 0.f;
-          V[r * kDVS + cc0 + b] = bt[r] * (vv - eg[r] * acc[aa][b]);
+        for (int e = 0; e < 4; ++e) {
+          const int r = vr0 + g8 + 8 * (e >> 1), cc = vc0 + 8 * jj + 2 * t4 + (e & 1);
+          const int64_t tk = c0 + r;
+          const float vv = tk < seq_end ? to_f32(v[((size_t)tk * nv + h) * dv + cslice + cc]) : 0.f;
+          V[r * kDVS + cc] = bt[r] * (vv - eg[r] * acc[jj][e]);
         }
-      }
     }
     __syncthreads();
-    // ---- V' = T X = X + (T - I) X  (one 4x4 tile per thread: NTV <= kThreads) ----
+    // ---- V' = T X = X + (T - I) X  (T - I is zero from the diagonal up) ----
     {
-      static_assert(NTV <= kThreads, "one V' tile per thread");
-      float acc[4][4];
-      const int r0 = (tid / (kDVS / 4)) * 4, cc0 = (tid % (kDVS / 4)) * 4;
-      if (tid < NTV) {
+      float acc[NTV][4] = {};
+      warp_mma_3xtf32<NTV>(acc, 0, vr0 + 16,
+                           [&](int m, int kk) { return A[(vr0 + m) * L::AP + kk]; },
+                           [&](int kk, int n) { return V[kk * kDVS + vc0 + n]; }, g8, t4);
+      __syncthreads();  // every warp has read X
 #pragma unroll
-        for (int aa = 0; aa < 4; ++aa) {
-          const float4 x = *reinterpret_cast<const float4*>(V + (r0 + aa) * kDVS + cc0);
-          acc[aa][0] = x.x; acc[aa][1] = x.y; acc[aa][2] = x.z; acc[aa][3] = x.w;
+      for (int jj = 0; jj < NTV; ++jj)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int r = vr0 + g8 + 8 * (e >> 1), cc = vc0 + 8 * jj + 2 * t4 + (e & 1);
+          V[r * kDVS + cc] += acc[jj][e];
         }
-        for (int i = 0; i < r0 + 3; ++i) {
-          const float4 y = *reinterpret_cast<const float4*>(V + i * kDVS + cc0);
-          const float ys[4] = {y.x, y.y, y.z, y.w};
-#pragma unroll
-          for (int aa = 0; aa < 4; ++aa) {
-            const float t_ri = A[(r0 + aa) * L::AP + i];  // zero for i >= r
-#pragma unroll
-            for (int b = 0; b < 4; ++b) acc[aa][b] = fmaf(t_ri, ys[b], acc[aa][b]);
-          }
-        }
-      }
-      __syncthreads();
-      if (tid < NTV) {
-#pragma unroll
-        for (int aa = 0; aa < 4; ++aa)
-          *reinterpret_cast<float4*>(V + (r0 + aa) * kDVS + cc0) =
-              make_float4(acc[aa][0], acc[aa][1], acc[aa][2], acc[aa][3]);
-      }
     }
     __syncthreads();
     // ---- P = (Q K^T * Gamma), lower including the diagonal ----
     pair_matrix<C, DK, true>(sm, tid);
     __syncthreads();
-    // ---- o = diag(exp(gcum)) Q S + P V' ----
-    for (int tile = tid; tile < NTV; tile += kThreads) {
-      const int r0 = (tile / (kDVS / 4)) * 4, cc0 = (tile % (kDVS / 4)) * 4;
-      float acc[4][4] = {};
-#pragma unroll 4
-      for (int d = 0; d < DK; ++d) {
-        const float4 x = ld4_t<C>(QhT, d, r0);
-        const float4 y = *reinterpret_cast<const float4*>(S + d * kDVS + cc0);
-        const float xs[4] = {x.x, x.y, x.z, x.w};
-        const float ys[4] = {y.x, y.y, y.z, y.w};
+    // ---- o = diag(exp(gcum)) Q S + P V'  (P is zero above the diagonal) ----
+    {
+      float qs[NTV][4] = {}, pv[NTV][4] = {};
+      warp_mma_3xtf32<NTV>(qs, 0, DK,
+                           [&](int m, int kk) { return QhT[swz<C>(kk, vr0 + m)]; },
+                           [&](int kk, int n) { return S[kk * kDVS + vc0 + n]; }, g8, t4);
+      warp_mma_3xtf32<NTV>(pv, 0, vr0 + 16,
+                           [&](int m, int kk) { return A[(vr0 + m) * L::AP + kk]; },
+                           [&](int kk, int n) { return V[kk * kDVS + vc0 + n]; }, g8, t4);
 #pragma unroll
-        for (int aa = 0; aa < 4; ++aa)
+      for (int jj = 0; jj < NTV; ++jj)
 #pragma unroll
-          for (int b = 0; b < 4; ++b) acc[aa][b] = fmaf(xs[aa], ys[b], acc[aa][b]);
-      }
-#pragma unroll
-      for (int aa = 0; aa < 4; ++aa)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) acc[aa][b] *= eg[r0 + aa];
-      for (int i = 0; i <= r0 + 3 && i < C; ++i) {
-        const float4 y = *reinterpret_cast<const float4*>(V + i * kDVS + cc0);
-        const float ys[4] = {y.x, y.y, y.z, y.w};
-#pragma unroll
-        for (int aa = 0; aa < 4; ++aa) {
-          const float p = A[(r0 + aa) * L::AP + i];  // zero for i > r
-#pragma unroll
-          for (int b = 0; b < 4; ++b) acc[aa][b] = fmaf(p, ys[b], acc[aa][b]);
+        for (int e = 0; e < 4; ++e) {
+          const int r = vr0 + g8 + 8 * (e >> 1), cc = vc0 + 8 * jj + 2 * t4 + (e & 1);
+          const int64_t tk = c0 + r;
+          if (tk < seq_end)
+            out[((size_t)tk * nv + h) * dv + cslice + cc] = from_f32<IO>(fmaf(eg[r], qs[jj][e], pv[jj][e]));
         }
-      }
-#pragma unroll
-      for (int aa = 0; aa < 4; ++aa) {
-        const int64_t t = c0 + r0 + aa;
-        if (t < seq_end) {
-          IO* orow = out + ((size_t)t * nv + h) * dv + cslice + cc0;
-#pragma unroll
-          for (int b = 0; b < 4; ++b) orow[b] = from_f32<IO>(acc[aa][b]);
-        }
-      }
     }
     __syncthreads();
     // ---- S <- exp(g_last) S + (K * exp(g_last - gcum))^T V' ----
     {
       const float decay = expf(gc[C - 1]);
-      constexpr int NTS = (DK / 4) * (kDVS / 4);
-      for (int tile = tid; tile < NTS; tile += kThreads) {
-        const int d0 = (tile / (kDVS / 4)) * 4, cc0 = (tile % (kDVS / 4)) * 4;
-        float acc[4][4] = {};
-        for (int r = 0; r < C; ++r) {
-          const float w = ekl[r];
-          const float4 y = *reinterpret_cast<const float4*>(V + r * kDVS + cc0);
-          const float ys[4] = {y.x * w, y.y * w, y.z * w, y.w * w};
+      const int sr0 = 16 * ((warp * NTS) / 4), sc0 = 8 * ((warp * NTS) % 4);
+      float acc[NTS][4] = {};
+      warp_mma_3xtf32<NTS>(acc, 0, C,
+                           [&](int m, int kk) { return KhT[swz<C>(sr0 + m, kk)]; },
+                           [&](int kk, int n) { return ekl[kk] * V[kk * kDVS + sc0 + n]; }, g8, t4);
 #pragma unroll
-          for (int aa = 0; aa < 4; ++aa) {
-            const float kk = KhT[swz<C>(d0 + aa, r)];
+      for (int jj = 0; jj < NTS; ++jj)
 #pragma unroll
-            for (int b = 0; b < 4; ++b) acc[aa][b] = fmaf(kk, ys[b], acc[aa][b]);
-          }
+        for (int e = 0; e < 4; ++e) {
+          const int d = sr0 + g8 + 8 * (e >> 1), cc = sc0 + 8 * jj + 2 * t4 + (e & 1);
+          S[d * kDVS + cc] = fmaf(S[d * kDVS + cc], decay, acc[jj][e]);
         }
-#pragma unroll
-        for (int aa = 0; aa < 4; ++aa) {
-          float4* sp = reinterpret_cast<float4*>(S + (d0 + aa) * kDVS + cc0);
-          float4 s = *sp;
-          s.x = fmaf(s.x, decay, acc[aa][0]);
-          s.y = fmaf(s.y, decay, acc[aa][1]);
-          s.z = fmaf(s.z, decay, acc[aa][2]);
-          s.w = fmaf(s.w, decay, acc[aa][3]);
-          *sp = s;
-        }
-      }
     }
   }
   __syncthreads();
