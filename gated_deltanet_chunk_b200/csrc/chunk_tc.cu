@@ -573,42 +573,54 @@ __global__ void __launch_bounds__(kThreads, 1)
         spp[SP_SQ + t] = si[SI_SQ + t];
         if (t == 0) spp[SP_GAMMA] = si[SI_GAM];
       }
-      if (krow) {  // (P was stored while the diagonal blocks were solved)
-        uint4 pk1[4];
-        float x[32];  // row r of T, columns [c0, c0 + 32)
-        if (r < 32 && hf == 1) {
+      {
+        // every thread a quarter row of T (row pr, columns [16 qc, 16 qc + 16));
+        // P was stored while the diagonal blocks were solved
+        const int pr = t & 63, qc = t >> 6, ph = qc >> 1, sub = qc & 1;
+        float x[16];
+        if (pr < 32 && ph == 1) {
 #pragma unroll
-          for (int cc = 0; cc < 32; ++cc) x[cc] = 0.f;
+          for (int cc = 0; cc < 16; ++cc) x[cc] = 0.f;
         } else {
-          const float* tr = ms + (r < 32 ? r * MS_LD : (hf == 0 ? (r - 32) * MS_LD + 32 : r * MS_LD + 32));
+          const float* tr =
+              ms + (pr < 32 ? pr * MS_LD : (ph == 0 ? (pr - 32) * MS_LD + 32 : pr * MS_LD + 32)) + 16 * sub;
 #pragma unroll
-          for (int v = 0; v < 8; ++v) {
+          for (int v = 0; v < 4; ++v) {
             const float4 y = *reinterpret_cast<const float4*>(tr + 4 * v);
             x[4 * v] = y.x; x[4 * v + 1] = y.y; x[4 * v + 2] = y.z; x[4 * v + 3] = y.w;
           }
-          if ((r >> 5) == hf) {  // a diagonal 32 x 32 block: T is zero above the diagonal
-            const int rl = r & 31;
+          if ((pr >> 5) == ph) {  // a diagonal 32 x 32 block: T is zero above the diagonal
+            const int lim = (pr & 31) - 16 * sub;
 #pragma unroll
-            for (int cc = 0; cc < 32; ++cc) x[cc] = cc <= rl ? x[cc] : 0.f;
+            for (int cc = 0; cc < 16; ++cc) x[cc] = cc <= lim ? x[cc] : 0.f;
           }
         }
-        float y[32];
+        float y[16];
+        uint4 wv[2], tu[2];
 #pragma unroll
-        for (int cc = 0; cc < 32; ++cc) y[cc] = -x[cc] * si[SI_BW + c0 + cc];
-        ptx::pack_half_bf16(y, pk0);  // -T diag(beta exp(gcum) rk), for W
-        ptx::st_half_packed(ps + PS_WHI, r, hf, pk0);
+        for (int cc = 0; cc < 16; ++cc) y[cc] = -x[cc] * si[SI_BW + 16 * qc + cc];
+        wv[0] = ptx::pack8_bf16(y);  // -T diag(beta exp(gcum) rk), for W
+        wv[1] = ptx::pack8_bf16(y + 8);
 #pragma unroll
-        for (int cc = 0; cc < 32; ++cc) y[cc] = x[cc] * si[SI_BETA + c0 + cc];
-        ptx::pack_half_bf16(y, pk1);  // T diag(beta), for U
-        ptx::st_half_packed(ps + PS_TU, r, hf, pk1);
+        for (int cc = 0; cc < 16; ++cc) y[cc] = x[cc] * si[SI_BETA + 16 * qc + cc];
+        tu[0] = ptx::pack8_bf16(y);  // T diag(beta), for U
+        tu[1] = ptx::pack8_bf16(y + 8);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          *reinterpret_cast<uint4*>(ps + PS_WHI + ptx::sw128_off(pr, 2 * qc + c)) = wv[c];
+          *reinterpret_cast<uint4*>(ps + PS_TU + ptx::sw128_off(pr, 2 * qc + c)) = tu[c];
+        }
         ptx::fence_proxy_async_smem();
         if (t < 64) {
           ptx::st_async_b32(rspp + 4 * (SP_WK + t), __float_as_uint(si[SI_WK + t]), rbar);
           ptx::st_async_b32(rspp + 4 * (SP_SQ + t), __float_as_uint(si[SI_SQ + t]), rbar);
           if (t == 0) ptx::st_async_b32(rspp + 4 * SP_GAMMA, __float_as_uint(si[SI_GAM]), rbar);
         }
-        ptx::st_half_packed_remote(rpa + PS_WHI, rbar, r, hf, pk0);
-        ptx::st_half_packed_remote(rpa + PS_TU, rbar, r, hf, pk1);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          ptx::st_async_v4(rpa + PS_WHI + ptx::sw128_off(pr, 2 * qc + c), wv[c], rbar);
+          ptx::st_async_v4(rpa + PS_TU + ptx::sw128_off(pr, 2 * qc + c), tu[c], rbar);
+        }
       }
       named_bar_n(1, 256);
       if (t == 0) ptx::mbar_arrive(bars + BAR_PRODF + psl);  // the other CTA's copy completes by transactions
