@@ -253,13 +253,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < 8) {
     // =====================================================================
     // intra warps (0-7): thread (quarter q = warp % 4, half h = warp / 4, lane)
-    // owns columns [32h, 32h + 32) of accumulator row 32q + lane.
+    // owns accumulator row 32q + lane of G, columns [16h, 16h + 16) and
+    // [32 + 16h, 48 + 16h).
     // =====================================================================
     const int t = tid;  // 0..255
     const int q = warp & 3, hf = warp >> 2;
     const int row = 32 * q + lane;  // accumulator row: 0..63 keys, 64..127 queries
     const int r = row & 63;
-    const int c0 = 32 * hf;
     const bool krow = q < 2;
     float* ms = reinterpret_cast<float*>(sm + OFF_MS);
     uint32_t ph_mma = 0;
@@ -362,55 +362,68 @@ __global__ void __launch_bounds__(kThreads, 1)
       // (query rows) wait in registers, packed to bf16, until the slot is free
       uint4 pk0[4];
       {
-        // G row r, columns [c0, c0 + 32), scaled to A (key rows) or P (query rows):
+        // G row r, scaled to A (key rows) or P (query rows):
         //   A[r][i] = -beta_r rk_r rk_i exp(gcum_r - gcum_i) (K K^T)[r][i],  i < r
         //   P[r][i] =  rq_r rk_i exp(gcum_r - gcum_i) (Q K^T)[r][i],        i <= r
-        // The decay is formed only where i <= r (mask before exp).  In a half that
-        // lies wholly below row r it is split at the half's last column b,
-        // exp(gcum_r - gcum_b) exp(gcum_b - gcum_i), both factors <= 1 for gates <= 0.
+        // The thread takes 16 columns from each 32-column block, [16 hf, 16 hf + 16)
+        // and [32 + 16 hf, 48 + 16 hf), so every warp has one 16-column run in its
+        // rows' diagonal block.  The decay is formed only where i <= r (mask before
+        // exp); for a run in the block left of the diagonal block (rows 32..63,
+        // columns < 32) it is split at column 31, exp(gcum_r - gcum_31)
+        // exp(gcum_31 - gcum_i), both factors <= 1 for gates <= 0.
         float av[32];
-        ptx::tmem_ld32(tl + TM_G + c0, av);
+        ptx::tmem_ld16(tl + TM_G + 16 * hf, av);
+        ptx::tmem_ld16(tl + TM_G + 32 + 16 * hf, av + 16);
         ptx::tmem_ld_wait();
         ptx::tc_fence_before();  // G is consumed: the next chunk's G may overwrite it after any barrier
         const float f = krow ? -si[SI_BETA + r] * si[SI_RK + r] : si[SI_RQ + r];
         const int rblk = r >> 5;  // == q & 1: warp-uniform
-        if (rblk > hf) {
-          const float rowf = f * fast_exp(si[SI_GC + r] - si[SI_GC + c0 + 31]);
-          const float4* cf = reinterpret_cast<const float4*>(si + SI_CF + c0);
+        // the run in the diagonal block, columns [cd, cd + 16) (both branches below
+        // index av with constants, keeping it in registers)
+        auto diag_run = [&](float* dg, int cd) {
+          const float gr = si[SI_GC + r];
+          const int lim = krow ? r : r + 1;  // columns i < lim are kept
+          const float4* rk4 = reinterpret_cast<const float4*>(si + SI_RK + cd);
+          const float4* gc4 = reinterpret_cast<const float4*>(si + SI_GC + cd);
 #pragma unroll
-          for (int k4 = 0; k4 < 8; ++k4) {
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const float4 rk = rk4[k4], gc = gc4[k4];
+            const int i0 = cd + 4 * k4;
+            dg[4 * k4 + 0] = (i0 + 0 < lim) ? dg[4 * k4 + 0] * (f * rk.x) * fast_exp(gr - gc.x) : 0.f;
+            dg[4 * k4 + 1] = (i0 + 1 < lim) ? dg[4 * k4 + 1] * (f * rk.y) * fast_exp(gr - gc.y) : 0.f;
+            dg[4 * k4 + 2] = (i0 + 2 < lim) ? dg[4 * k4 + 2] * (f * rk.z) * fast_exp(gr - gc.z) : 0.f;
+            dg[4 * k4 + 3] = (i0 + 3 < lim) ? dg[4 * k4 + 3] * (f * rk.w) * fast_exp(gr - gc.w) : 0.f;
+          }
+        };
+        if (rblk == 1) {
+          const float rowf = f * fast_exp(si[SI_GC + r] - si[SI_GC + 31]);
+          const float4* cf = reinterpret_cast<const float4*>(si + SI_CF + 16 * hf);
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4) {
             const float4 x = cf[k4];
             av[4 * k4 + 0] *= rowf * x.x;
             av[4 * k4 + 1] *= rowf * x.y;
             av[4 * k4 + 2] *= rowf * x.z;
             av[4 * k4 + 3] *= rowf * x.w;
           }
-        } else if (rblk == hf) {
-          const float gr = si[SI_GC + r];
-          const int lim = krow ? r : r + 1;  // columns i < lim are kept
-          const float4* rk4 = reinterpret_cast<const float4*>(si + SI_RK + c0);
-          const float4* gc4 = reinterpret_cast<const float4*>(si + SI_GC + c0);
-#pragma unroll
-          for (int k4 = 0; k4 < 8; ++k4) {
-            const float4 rk = rk4[k4], gc = gc4[k4];
-            const int i0 = c0 + 4 * k4;
-            av[4 * k4 + 0] = (i0 + 0 < lim) ? av[4 * k4 + 0] * (f * rk.x) * fast_exp(gr - gc.x) : 0.f;
-            av[4 * k4 + 1] = (i0 + 1 < lim) ? av[4 * k4 + 1] * (f * rk.y) * fast_exp(gr - gc.y) : 0.f;
-            av[4 * k4 + 2] = (i0 + 2 < lim) ? av[4 * k4 + 2] * (f * rk.z) * fast_exp(gr - gc.z) : 0.f;
-            av[4 * k4 + 3] = (i0 + 3 < lim) ? av[4 * k4 + 3] * (f * rk.w) * fast_exp(gr - gc.w) : 0.f;
-          }
+          diag_run(av + 16, 32 + 16 * hf);
         } else {
+          diag_run(av, 16 * hf);
 #pragma unroll
-          for (int cc = 0; cc < 32; ++cc) av[cc] = 0.f;
+          for (int cc = 16; cc < 32; ++cc) av[cc] = 0.f;  // above the diagonal block
         }
         if (krow) {
-          if (rblk >= hf) {  // the 32 x 32 block above the diagonal is zero and never read
-            float* mc = ms + c0 * MS_LD + r;  // M[i][r] = A[r][i]: column i of A is row i of M
+          // M[i][r] = A[r][i] (column i of A is row i of M); the 32 x 32 block above
+          // the diagonal is zero and never read
+          float* mc = ms + 16 * hf * MS_LD + r;
 #pragma unroll
-            for (int cc = 0; cc < 32; ++cc) mc[cc * MS_LD] = av[cc];
+          for (int cc = 0; cc < 16; ++cc) mc[cc * MS_LD] = av[cc];
+          if (rblk == 1) {
+#pragma unroll
+            for (int cc = 0; cc < 16; ++cc) mc[(32 + cc) * MS_LD] = av[16 + cc];
           }
         } else {
-          ptx::pack_half_bf16(av, pk0);  // P
+          ptx::pack_half_bf16(av, pk0);  // P: chunks 2 hf, 2 hf + 1, 4 + 2 hf, 5 + 2 hf of the row
         }
       }
       // the product slot (both copies) must have been released by both CTAs'
@@ -471,9 +484,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 16; ++i) mb[i * MS_LD + lane] = x[i];  // T_bb, row-major
         }
       } else {
-        ptx::st_half_packed(ps + PS_P, r, hf, pk0);  // P
+#pragma unroll
+        for (int c = 0; c < 4; ++c)  // P
+          *reinterpret_cast<uint4*>(ps + PS_P + ptx::sw128_off(r, 2 * hf + (c & 1) + 4 * (c >> 1))) = pk0[c];
         ptx::fence_proxy_async_smem();
-        ptx::st_half_packed_remote(rpa + PS_P, rbar, r, hf, pk0);
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          ptx::st_async_v4(rpa + PS_P + ptx::sw128_off(r, 2 * hf + (c & 1) + 4 * (c >> 1)), pk0[c], rbar);
       }
       named_bar_n(1, 256);
       // 2. both 32 x 32 diagonal blocks: T_10 = T_11 (A_10 T_00) on 16 x 16 blocks,
