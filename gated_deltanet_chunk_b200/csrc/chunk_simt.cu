@@ -60,32 +60,6 @@ __device__ __forceinline__ float4 ld4_t(const float* base, int d, int r0) {
   return *reinterpret_cast<const float4*>(base + swz<C>(d, r0));
 }
 
-// PER consecutive elements of one row (from a 4 * PER-byte or 2 * PER-byte
-// aligned address) as fp32; zeros for a row past the sequence end.
-template <typename IO, int PER>
-__device__ __forceinline__ void load_row_part(const IO* p, bool valid, float* x) {
-  if (!valid) {
-#pragma unroll
-    for (int e = 0; e < PER; ++e) x[e] = 0.f;
-    return;
-  }
-  if constexpr (sizeof(IO) == 4 && PER == 4) {
-    const float4 y = *reinterpret_cast<const float4*>(p);
-    x[0] = y.x; x[1] = y.y; x[2] = y.z; x[3] = y.w;
-  } else if constexpr (sizeof(IO) == 4 && PER == 2) {
-    const float2 y = *reinterpret_cast<const float2*>(p);
-    x[0] = y.x; x[1] = y.y;
-  } else if constexpr (sizeof(IO) == 2 && PER == 4) {
-    const uint2 y = *reinterpret_cast<const uint2*>(p);
-    const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&y.x));
-    const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&y.y));
-    x[0] = lo.x; x[1] = lo.y; x[2] = hi.x; x[3] = hi.y;
-  } else {
-#pragma unroll
-    for (int e = 0; e < PER; ++e) x[e] = to_f32(p[e]);
-  }
-}
-
 // fp32 x = hi + lo with hi, lo both TF32 (the low 13 bits of each are zero):
 // products of such splits, hi hi + hi lo + lo hi, are within about 2^-22 of
 // the exact product, so three TF32 MMAs stand in for fp32 ones.  That is four
@@ -186,7 +160,7 @@ __device__ __forceinline__ void pair_matrix(float* sm, int tid) {
 //      and one column per lane: (T - I)[i][j] = A[i][j] + sum_{j<m<i} A[i][m] (T - I)[m][j];
 //   2. doubling the solved blocks, for s = 16, 32, ... < C: a diagonal block
 //      [[T00, 0], [T10, T11]] of size 2s has T10 = T11 A10 T00, formed as
-//      Y = A10 + A10 (T00 - I), then T10 = Y + (T11 - I) Y.
+//      Y = A10 + A10 (T00 - I), then T10 = Y + (T11 - I) Y (warp MMAs below).
 // Y needs s x s floats per pair (C s / 2 in all), held in the V tile, which
 // is free until X is formed.
 template <int C, int DK>
@@ -216,66 +190,48 @@ __device__ __forceinline__ void invert_blocked(float* sm, int tid) {
       if (jc < i) blk[i * AP + jc] = x[i];
   }
   __syncthreads();
+  // the doubling merges as warp MMAs (TF32 split three ways): a unit is one
+  // pair's 16 x 16 output block (two 16 x 8 tiles); phase 1 forms Y, phase 2 T10
 #pragma unroll 1
   for (int s = 16; s < C; s *= 2) {
-    // one 4 x 4 tile of the level's outputs per thread and pass
-    const int ts = s / 4, ntile = (C / (2 * s)) * ts * ts;
-    for (int e = tid; e < ntile; e += kThreads) {
-      const int p = e / (ts * ts), i0 = 4 * ((e / ts) % ts), j0 = 4 * (e % ts);
+    const int nb = s / 16, nunit = (C / (2 * s)) * nb * nb;
+    const int g = lane >> 2, t = lane & 3;
+    for (int u = warp; u < nunit; u += kThreads / 32) {
+      const int p = u / (nb * nb), rb = (u / nb) % nb, cb = u % nb;
       const int base = 2 * s * p;
-      const float* a10 = A + (base + s) * AP + base;  // A10[i][m] = a10[i * AP + m]
-      const float* t00 = A + base * AP + base;        // (T00 - I)[m][j], zero for m <= j
-      float acc[4][4];
-#pragma unroll
-      for (int r = 0; r < 4; ++r)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) acc[r][c] = a10[(i0 + r) * AP + j0 + c];
-#pragma unroll 4
-      for (int m = j0 + 1; m < s; ++m) {
-        float x[4], y[4];
-#pragma unroll
-        for (int r = 0; r < 4; ++r) x[r] = a10[(i0 + r) * AP + m];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) y[c] = t00[m * AP + j0 + c];
-#pragma unroll
-        for (int r = 0; r < 4; ++r)
-#pragma unroll
-          for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(x[r], y[c], acc[r][c]);
-      }
+      const float* a10 = A + (base + s + 16 * rb) * AP + base;  // rows 16 rb.. of A10
+      const float* t00 = A + base * AP + base + 16 * cb;         // (T00 - I), columns 16 cb..
+      float acc[2][4] = {};
+      // (T00 - I)[k][j] is zero for k <= j: k starts at the column block
+      warp_mma_3xtf32<2>(acc, 16 * cb, s, [&](int m, int kk) { return a10[m * AP + kk]; },
+                         [&](int kk, int n) { return t00[kk * AP + n]; }, g, t);
       float* yp = Y + p * s * s;
 #pragma unroll
-      for (int r = 0; r < 4; ++r)
-        *reinterpret_cast<float4*>(yp + (i0 + r) * s + j0) = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+      for (int jj = 0; jj < 2; ++jj)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int m = 16 * rb + g + 8 * (e >> 1), jc = 16 * cb + 8 * jj + 2 * t + (e & 1);
+          yp[m * s + jc] = a10[(g + 8 * (e >> 1)) * AP + jc] + acc[jj][e];
+        }
     }
     __syncthreads();
-    for (int e = tid; e < ntile; e += kThreads) {
-      const int p = e / (ts * ts), i0 = 4 * ((e / ts) % ts), j0 = 4 * (e % ts);
+    for (int u = warp; u < nunit; u += kThreads / 32) {
+      const int p = u / (nb * nb), rb = (u / nb) % nb, cb = u % nb;
       const int base = 2 * s * p;
-      const float* t11 = A + (base + s) * AP + base + s;  // (T11 - I)[i][m], zero for m >= i
+      const float* t11 = A + (base + s + 16 * rb) * AP + base + s;  // rows 16 rb.. of (T11 - I)
       const float* yp = Y + p * s * s;
-      float acc[4][4];
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const float4 y = *reinterpret_cast<const float4*>(yp + (i0 + r) * s + j0);
-        acc[r][0] = y.x; acc[r][1] = y.y; acc[r][2] = y.z; acc[r][3] = y.w;
-      }
-#pragma unroll 4
-      for (int m = 0; m < i0 + 3; ++m) {
-        float x[4];
-#pragma unroll
-        for (int r = 0; r < 4; ++r) x[r] = t11[(i0 + r) * AP + m];
-        const float4 y = *reinterpret_cast<const float4*>(yp + m * s + j0);
-        const float yv[4] = {y.x, y.y, y.z, y.w};
-#pragma unroll
-        for (int r = 0; r < 4; ++r)
-#pragma unroll
-          for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(x[r], yv[c], acc[r][c]);
-      }
+      float acc[2][4] = {};
+      // (T11 - I)[i][m] is zero for m >= i: columns up to the row block's end
+      warp_mma_3xtf32<2>(acc, 0, 16 * rb + 16, [&](int m, int kk) { return t11[m * AP + kk]; },
+                         [&](int kk, int n) { return yp[kk * s + 16 * cb + n]; }, g, t);
       float* t10 = A + (base + s) * AP + base;
 #pragma unroll
-      for (int r = 0; r < 4; ++r)
+      for (int jj = 0; jj < 2; ++jj)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) t10[(i0 + r) * AP + j0 + c] = acc[r][c];
+        for (int e = 0; e < 4; ++e) {
+          const int m = 16 * rb + g + 8 * (e >> 1), jc = 16 * cb + 8 * jj + 2 * t + (e & 1);
+          t10[m * AP + jc] = yp[m * s + jc] + acc[jj][e];
+        }
     }
     __syncthreads();
   }
@@ -329,9 +285,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_simt_kernel(ChunkArgs a
       for (int rb = 0; rb < RB; ++rb) {
         const int64_t t = c0 + r0 + rb;
         const bool valid = t < seq_end;
-        const size_t off = ((size_t)(valid ? t : 0) * nqk + j) * DK + lane * PER;
-        load_row_part<IO, PER>(q + off, valid, qv[rb]);
-        load_row_part<IO, PER>(k + off, valid, kv[rb]);
+        // lane l holds elements l, l + 32, ...: each load is one coalesced row
+        // segment, and the transposed stores below spread over the banks
+        const size_t off = ((size_t)(valid ? t : 0) * nqk + j) * DK + lane;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) {
+          qv[rb][e] = valid ? to_f32(q[off + 32 * e]) : 0.f;
+          kv[rb][e] = valid ? to_f32(k[off + 32 * e]) : 0.f;
+        }
       }
 #pragma unroll
       for (int rb = 0; rb < RB; ++rb) {
@@ -357,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_simt_kernel(ChunkArgs a
         const float fk = a.qk_l2norm ? 1.f / sqrtf(sk[rb] + kNormEps) : 1.f;
 #pragma unroll
         for (int e = 0; e < PER; ++e) {
-          const int d = lane * PER + e;
+          const int d = 32 * e + lane;
           QhT[swz<C>(d, r)] = qv[rb][e] * fq;
           KhT[swz<C>(d, r)] = kv[rb][e] * fk;
         }
