@@ -56,7 +56,12 @@ typedef enum {
 typedef enum { GDN_DTYPE_F32 = 0, GDN_DTYPE_BF16 = 1 } gdn_dtype_t;
 
 /* Kernel family for gdn_chunk_fwd.  AUTO picks the tensor-core kernel where it
- * applies (bf16 io, Dk = Dv = 128) and the SIMT kernel otherwise. */
+ * applies (bf16 io, Dk = Dv = 128, chunk_size 64) and the SIMT kernel
+ * otherwise: fp32 io, Dk or Dv = 64, or chunk_size 128.  The SIMT kernel keeps
+ * fp32 accuracy (fp32 FMAs, and warp-level TF32 MMAs with each operand split
+ * into two TF32 parts) and is several times slower per token; since the result
+ * does not depend on chunk_size beyond rounding, bf16 callers get the fast path
+ * with chunk_size 64. */
 typedef enum { GDN_KERNEL_AUTO = 0, GDN_KERNEL_SIMT = 1, GDN_KERNEL_TC = 2 } gdn_kernel_t;
 
 /* Shapes and options shared by both calls. */
